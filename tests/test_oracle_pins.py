@@ -1,0 +1,282 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle.
+
+* the spectral closed form of an odd matrix polynomial (textbook SVD):
+  NS_T(X) = U diag(f(sigma)) V^T with f the scalar quintic iterated T times;
+* the Gram rewrite p(t) = t q(t^2) (Gram Newton-Schulz page, section on the
+  algorithm's advantage): the Gram iteration equals the standard one;
+* the coefficient claims of the NanoGPT/Muon page (section on coefficient
+  tuning): (2, -1.5, 0.5) converges to polar(X) = U V^T, the tuned set lands
+  singular values in roughly [0.7, 1.3] after five steps;
+* the ROOT page's worked number (golden file): MSE 0.0499 on 2048 x 2048;
+* the closed form of SGD momentum under a constant gradient;
+* invariances (transpose, positive scale) and special cases (zero input,
+  zero steps).
+
+The last block plants plausible mistakes in copies of the oracle and checks
+that these pins catch every one of them.
+"""
+import os
+
+import numpy as np
+import pytest
+
+from oracle import muon_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _scalar_f(sigma, coeffs, steps):
+    """f = p_T o ... o p_1 applied to scalars, p_k(s) = a s + b s^3 + c s^5."""
+    s = np.array(sigma, dtype=np.float64)
+    for a, b, c in orc._coeff_list(coeffs, steps):
+        s = a * s + b * s ** 3 + c * s ** 5
+    return s
+
+
+def _spectral_ns(X, coeffs, steps):
+    U, S, Vt = np.linalg.svd(X, full_matrices=False)
+    return (U * _scalar_f(S, coeffs, steps)) @ Vt
+
+
+def _relF(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+SHAPES = [(24, 40), (32, 32), (40, 24), (7, 61)]
+COEFFS = [orc.TUNED_COEFFS, orc.BASELINE_COEFFS,
+          # per-step coefficients (one triple per step)
+          ((3.4445, -4.7750, 2.0315), (2.9, -4.0, 1.9), (2.5, -3.0, 1.4),
+           (2.0, -1.5, 0.5), (1.875, -1.25, 0.375))]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("coeffs", COEFFS)
+@pytest.mark.parametrize("form", ["standard", "gram"])
+def test_ns_matches_spectral_closed_form(shape, coeffs, form):
+    X = _rng(1).standard_normal(shape)
+    X0 = X / (np.linalg.norm(X) + orc.DEFAULT_EPS)
+    got = orc.orthogonalize(X, coeffs, 5, form)
+    want = _spectral_ns(X0, coeffs, 5)
+    assert _relF(got, want) < 1e-11
+
+
+@pytest.mark.parametrize("restarts", [(), (1,), (2,), (3,), (2, 3), (1, 2, 3, 4)])
+@pytest.mark.parametrize("steps", [1, 2, 5, 7])
+def test_gram_equals_standard(restarts, steps):
+    X = _rng(2).standard_normal((20, 52))
+    X /= np.linalg.norm(X)
+    std = orc.ns_standard(X, orc.TUNED_COEFFS, steps)
+    gram = orc.ns_gram(X, orc.TUNED_COEFFS, steps, restarts)
+    assert _relF(gram, std) < 1e-12
+
+
+def test_baseline_coefficients_converge_to_polar():
+    X = _rng(3).standard_normal((48, 80))
+    U, S, Vt = np.linalg.svd(X, full_matrices=False)
+    # spread the singular values over [1e-3, 1] to exercise the slow end
+    S = np.geomspace(1e-3, 1.0, S.size)[::-1]
+    X = (U * S) @ Vt
+    polar = U @ Vt
+    for form in ("standard", "gram"):
+        got = orc.orthogonalize(X, orc.BASELINE_COEFFS, 40, form,
+                                restarts=(10, 20, 30))
+        assert np.max(np.abs(got - polar)) < 1e-10
+        sv = np.linalg.svd(got, compute_uv=False)
+        assert np.max(np.abs(sv - 1.0)) < 1e-10
+
+
+def test_tuned_coefficients_range():
+    """Five tuned steps send every singular value in [3e-3, 1] into about
+    [0.68, 1.21]; the page rounds this to [0.7, 1.3]."""
+    grid = np.linspace(3e-3, 1.0, 200001)
+    f = _scalar_f(grid, orc.TUNED_COEFFS, 5)
+    lo, hi = f.min(), f.max()
+    assert 0.66 < lo < 0.70 and 1.15 < hi < 1.30
+    for shape, dist in [((64, 256), "gauss"), ((128, 128), "gauss"),
+                        ((96, 300), "t3")]:
+        r = _rng(4)
+        X = r.standard_normal(shape) if dist == "gauss" else r.standard_t(3, shape)
+        X0 = X / np.linalg.norm(X)
+        smin = np.linalg.svd(X0, compute_uv=False).min()
+        out = orc.orthogonalize(X, orc.TUNED_COEFFS, 5, "standard")
+        sv = np.linalg.svd(out, compute_uv=False)
+        if smin >= 3e-3:
+            assert sv.min() >= lo - 1e-9 and sv.max() <= hi + 1e-9
+
+
+def _read_golden(name):
+    vals = {}
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                k, v = line.split()
+                vals[k] = float(v)
+    return vals
+
+
+def test_root_page_mse_2048():
+    g = _read_golden("root_orthogonality_mse.txt")
+    rows, cols = int(g["rows"]), int(g["cols"])
+    X = _rng(0).standard_normal((rows, cols))
+    out = orc.orthogonalize(X, (g["a"], g["b"], g["c"]), int(g["steps"]),
+                            "standard")
+    sv = np.linalg.svd(out, compute_uv=False)
+    mse = float(np.mean((sv - 1.0) ** 2))
+    assert abs(mse - g["mse"]) < g["tol"], mse
+
+
+def test_momentum_closed_form():
+    G = _rng(5).standard_normal((6, 9))
+    mu = 0.95
+    M = np.zeros_like(G)
+    for t in range(1, 12):
+        M, U = orc.momentum_update(M, G, mu, nesterov=True)
+        Mt = G * (1 - mu ** t) / (1 - mu)
+        assert np.allclose(M, Mt, rtol=1e-13, atol=0)
+        assert np.allclose(U, G + mu * Mt, rtol=1e-13, atol=0)
+    M2, U2 = orc.momentum_update(M, G, mu, nesterov=False)
+    assert np.array_equal(U2, M2)
+
+
+def test_transpose_equivariance():
+    X = _rng(6).standard_normal((30, 70))
+    for form in ("standard", "gram"):
+        a = orc.orthogonalize(X, steps=5, form=form)
+        b = orc.orthogonalize(X.T.copy(), steps=5, form=form)
+        assert _relF(b, a.T) < 1e-13
+
+
+def test_scale_invariance():
+    X = _rng(7).standard_normal((16, 40))
+    # exact invariance holds with eps = 0 (eps / ||X|| differs between scales)
+    a = orc.orthogonalize(X, form="standard", eps=0.0)
+    b = orc.orthogonalize(37.5 * X, form="standard", eps=0.0)
+    assert _relF(a, b) < 1e-12
+
+
+def test_zero_and_zero_steps():
+    Z = np.zeros((8, 12))
+    assert np.array_equal(orc.orthogonalize(Z, form="gram"), Z)
+    assert np.array_equal(orc.orthogonalize(Z, form="standard"), Z)
+    X = _rng(8).standard_normal((8, 12))
+    want = X / (np.linalg.norm(X) + orc.DEFAULT_EPS)
+    for form in ("standard", "gram"):
+        assert np.allclose(orc.orthogonalize(X, steps=0, form=form), want,
+                           rtol=1e-15, atol=0)
+
+
+def test_muon_step_update():
+    r = _rng(9)
+    W, G, M = (r.standard_normal((10, 14)) for _ in range(3))
+    W1, M1, O = orc.muon_step(W, G, M, mu=0.9, nesterov=True, lr=0.01,
+                              form="gram")
+    assert np.allclose(M1, 0.9 * M + G)
+    U = G + 0.9 * M1
+    assert _relF(O, _spectral_ns(U / (np.linalg.norm(U) + 1e-7),
+                                 orc.TUNED_COEFFS, 5)) < 1e-11
+    assert np.allclose(W1, W - 0.01 * O)
+
+
+def test_flop_formulas():
+    n, m = 96, 320
+    assert orc.ns_flops(n, m, 5, "standard") == 15 * n * n * m + 5 * n ** 3
+    assert orc.ns_flops(n, m, 5, "gram", ()) == 3 * n * n * m + 17 * n ** 3
+    assert orc.ns_flops(n, m, 5, "gram", (2,)) == 6 * n * n * m + 14 * n ** 3
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: each mutant is the oracle with one plausible error; the
+# pins above must reject all of them.
+
+def _mut_std_sign(X, coeffs, steps):
+    X = X.copy()
+    for a, b, c in orc._coeff_list(coeffs, steps):
+        A = X @ X.T
+        X = a * X + (-b * A + c * (A @ A)) @ X
+    return X
+
+
+def _mut_std_dropped_term(X, coeffs, steps):
+    X = X.copy()
+    for a, b, c in orc._coeff_list(coeffs, steps):
+        A = X @ X.T
+        X = a * X + (b * A) @ X
+    return X
+
+
+def _mut_std_transposed(X, coeffs, steps):
+    # multiplies q(X X^T) on the wrong side: X B instead of B X (square X)
+    X = X.copy()
+    for a, b, c in orc._coeff_list(coeffs, steps):
+        A = X @ X.T
+        B = b * A + c * (A @ A)
+        X = a * X + X @ B
+    return X
+
+
+def _mut_std_coeff_index(X, coeffs, steps):
+    X = X.copy()
+    for a, b, c in orc._coeff_list(coeffs, steps):
+        A = X @ X.T
+        X = a * X + (c * A + b * (A @ A)) @ X
+    return X
+
+
+def _mut_gram_no_right_z(X, coeffs, steps, restarts=(2,)):
+    X = X.copy()
+    n = X.shape[0]
+    I = np.eye(n)
+    R = X @ X.T
+    Q = I.copy()
+    for k, (a, b, c) in enumerate(orc._coeff_list(coeffs, steps)):
+        if k in restarts and k > 0:
+            X = Q @ X
+            R = X @ X.T
+            Q = I.copy()
+        Z = a * I + b * R + c * (R @ R)
+        Q = Z @ Q
+        R = Z @ R
+    return Q @ X
+
+
+def _mut_gram_restart_keeps_q(X, coeffs, steps, restarts=(2,)):
+    X = X.copy()
+    n = X.shape[0]
+    I = np.eye(n)
+    R = X @ X.T
+    Q = I.copy()
+    for k, (a, b, c) in enumerate(orc._coeff_list(coeffs, steps)):
+        if k in restarts and k > 0:
+            X = Q @ X
+            R = X @ X.T
+        Z = a * I + b * R + c * (R @ R)
+        Q = Z @ Q
+        R = Z @ R @ Z
+    return Q @ X
+
+
+@pytest.mark.parametrize("mutant", [_mut_std_sign, _mut_std_dropped_term,
+                                    _mut_std_transposed, _mut_std_coeff_index])
+def test_planted_standard_mistakes_are_caught(mutant):
+    X = _rng(1).standard_normal((32, 32))
+    X0 = X / (np.linalg.norm(X) + orc.DEFAULT_EPS)
+    want = _spectral_ns(X0, orc.TUNED_COEFFS, 5)
+    assert _relF(orc.ns_standard(X0, orc.TUNED_COEFFS, 5), want) < 1e-11
+    with np.errstate(over="ignore", invalid="ignore"):
+        bad = mutant(X0, orc.TUNED_COEFFS, 5)
+    err = _relF(bad, want) if np.all(np.isfinite(bad)) else np.inf
+    assert err > 1e-4
+
+
+@pytest.mark.parametrize("mutant", [_mut_gram_no_right_z,
+                                    _mut_gram_restart_keeps_q])
+def test_planted_gram_mistakes_are_caught(mutant):
+    X = _rng(2).standard_normal((20, 52))
+    X /= np.linalg.norm(X)
+    std = orc.ns_standard(X, orc.TUNED_COEFFS, 5)
+    assert _relF(mutant(X, orc.TUNED_COEFFS, 5), std) > 1e-4

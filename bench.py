@@ -1,0 +1,458 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 Muon optimizer step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ID]
+    python bench.py --impl reference ...      # the fp64 CPU oracle arm
+
+One step = one full Muon step over the workload's 2D parameters (momentum,
+Newton-Schulz, update) through the library's C ABI, or one batched
+orthogonalisation for the NS-only workloads.  Inputs are seeded synthetic
+tensors resident in HBM; the default workload (GPT-2 124M Muon set: 48
+matrices, 85 M elements, ~680 MB of params + grads + momentum per step) is
+larger than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own
+replica of the workload (weak scaling, no data-path collective) and the
+device time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from matrix_orthogonalizing_optimizer_step_b200 import workloads as wl  # noqa: E402
+
+METRIC = "Muon optimizer-step ms; Newton-Schulz bf16 TFLOP/s vs B200 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--form", default="auto", choices=["auto", "standard", "gram"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reported baseline; never part of the GPU path)
+
+def _ns_form_for(n, m, form):
+    from oracle import muon_oracle as orc
+    if form != "auto":
+        return form
+    return "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
+
+
+def cpu_oracle_step_ms(w, budget_s, form="auto"):
+    """Time the fp64 oracle on a bounded sample of one step of workload w and
+    scale to the whole step.  Matrices are taken in order (one of each shape
+    first) until the time budget is spent; the per-shape mean time is
+    multiplied by that shape's count."""
+    import numpy as np
+    import torch
+    from oracle import muon_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count() or 1
+    shapes = list(w.shapes)
+    order, seen = [], set()
+    for i, s in enumerate(shapes):
+        if s not in seen:
+            seen.add(s)
+            order.append(i)
+    order += [i for i in range(len(shapes)) if i not in set(order)]
+    per_shape = {}
+    t_start = time.perf_counter()
+    done = 0
+    for i in order:
+        if done and time.perf_counter() - t_start > budget_s and all(s in per_shape for s in seen):
+            break
+        r, c = shapes[i]
+        G = wl.make_matrix(w, i, wl.ROLE_GRAD).to(torch.float64).numpy()
+        n, m = min(r, c), max(r, c)
+        fm = _ns_form_for(n, m, form)
+        t0 = time.perf_counter()
+        if w.full_step:
+            M = wl.make_matrix(w, i, wl.ROLE_MOMENTUM).to(torch.float64).numpy()
+            W = wl.make_matrix(w, i, wl.ROLE_PARAM).to(torch.float64).numpy()
+            orc.muon_step(W, G, M, 0.95, True, 6e-4, form=fm)
+        else:
+            orc.orthogonalize(G, form=fm)
+        per_shape.setdefault((r, c), []).append(time.perf_counter() - t0)
+        done += 1
+    total_ms = 0.0
+    for s in seen:
+        cnt = sum(1 for x in shapes if x == s)
+        total_ms += 1e3 * statistics.fmean(per_shape[s]) * cnt
+    sample = (f"{done} of {len(shapes)} matrices (one of each of {len(seen)} shapes first), "
+              f"fp64 NumPy oracle, per-shape mean time x count")
+    return total_ms, cores, sample
+
+
+# ---------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid=None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:  # noqa: BLE001
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:  # noqa: BLE001
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 11:
+                    continue
+                if self.uuid and parts[1] != self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        load = [r for r in rows if (num(r[5]) or 0) > 10] or rows
+        sm = [num(r[2]) for r in load if num(r[2]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in load:
+            for name, v in zip(names, r[7:11]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][3]), "reasons": sorted(reasons),
+                "samples": len(load)}
+
+
+# ---------------------------------------------------------------------------
+
+def dist_setup(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def max_over_ranks(x, world, device=None):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def traffic_from_profiles(kernel_src):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    import hashlib
+    p = os.path.join(HERE, "profiles", "gemm_tc_gpt2_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as fh:
+        for line in fh:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    try:
+        with open(kernel_src, "rb") as fh:
+            h = hashlib.sha256(fh.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if vals.get("kernel_source_sha256_16") != h:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args):
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = wl.WORKLOADS[args.workload]
+    peaks, peak_src = load_peaks()
+
+    # ---- inputs (seeded, resident in HBM) --------------------------------
+    if w.full_step:
+        params = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=dev) for i in range(w.count)]
+        grads = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev) for i in range(w.count)]
+        moms = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
+        mo.muon_reset_config()
+        mo.muon_set_config(mode=args.form)
+
+        def step():
+            mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
+        bytes_in = sum(g.numel() * g.element_size() for g in grads)
+        in_bytes_resident = bytes_in + sum(p.numel() * p.element_size() for p in params) + \
+            sum(m.numel() * m.element_size() for m in moms)
+    else:
+        # NS-only workloads: one batched orthogonalisation per distinct shape
+        by_shape = {}
+        for i, s in enumerate(w.shapes):
+            by_shape.setdefault(s, []).append(i)
+        src = {s: torch.stack([wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev, dtype="bf16")
+                               for i in idx]) for s, idx in by_shape.items()}
+        work = {s: t.clone() for s, t in src.items()}
+
+        def step():
+            for s in work:
+                work[s].copy_(src[s])
+                mo.muon_orthogonalize(work[s], steps=5, mode=args.form)
+        bytes_in = sum(t.numel() * t.element_size() for t in src.values())
+        in_bytes_resident = 2 * bytes_in
+
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region --------------------------------------------------------
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001
+        pass
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+    mo.muon_profile_reset()
+    mo.muon_profile_enable(True)
+    launches0 = mo.muon_launch_count()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    launches = mo.muon_launch_count() - launches0
+    prof = mo.muon_profile_read()
+    mo.muon_profile_enable(False)
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_per_step = ms_total / args.steps
+
+    st, bad = mo.muon_device_status()
+    if st != mo.MUON_OK:
+        raise SystemExit(f"device status {mo.STATUS_NAMES.get(st, st)} (matrix {bad})")
+
+    # ---- roofline of the dominant kernel -------------------------------------
+    gemm = prof.get("gemm_tc", {})
+    momk = prof.get("momentum_norm", {})
+    gemm_tf = (gemm["flops"] / (gemm["total_ms"] * 1e-3) / 1e12) if gemm.get("total_ms") else 0.0
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    traffic = traffic_from_profiles(os.path.join(HERE, "matrix_orthogonalizing_optimizer_step_b200",
+                                                 "csrc", "gemm_tc.cu"))
+    roofline = {
+        "kernel": "gemm_tc (tcgen05 grouped GEMM, all Newton-Schulz products)",
+        "bound": "tensor", "achieved": round(gemm_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+        "frac": round(gemm_tf / peak_tf, 4) if peak_tf else None,
+        "traffic": traffic,
+        "peak_source": f"{peak_src} bf16_tflops (burst, cuBLAS); fp16 operands run at the same rate",
+        "launches": gemm.get("launches", 0), "avg_launch_ms": (gemm["total_ms"] / gemm["launches"]) if gemm.get("launches") else None,
+        "share_of_step": round(gemm.get("total_ms", 0) / ms_total, 4) if ms_total else None,
+    }
+    mom_gbs = (momk["bytes"] / (momk["total_ms"] * 1e-3) / 1e9) if momk.get("total_ms") else 0.0
+    peak_gbs = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    roofline_mom = {
+        "kernel": "momentum_norm (fused momentum/Nesterov/sum-of-squares/bf16 cast)",
+        "bound": "hbm", "achieved": round(mom_gbs, 1), "peak": peak_gbs, "unit": "GB/s",
+        "frac": round(mom_gbs / peak_gbs, 4) if peak_gbs else None,
+        "launches": momk.get("launches", 0),
+        "share_of_step": round(momk.get("total_ms", 0) / ms_total, 4) if ms_total else None,
+    }
+    ns_tflops = gemm.get("flops", 0) / (ms_total * 1e-3) / 1e12 if ms_total else 0.0
+
+    # ---- end to end through the public API, host buffers ---------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e_steps = max(1, min(args.steps, 10))
+        if w.full_step:
+            host_g = [g.detach().to("cpu").pin_memory() for g in grads]
+            host_p = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
+
+            def e2e_step():
+                for h, g in zip(host_g, grads):
+                    g.copy_(h, non_blocking=True)
+                step()
+                for h, p in zip(host_p, params):
+                    h.copy_(p, non_blocking=True)
+            h2d = bytes_in
+            d2h = sum(p.numel() * p.element_size() for p in params)
+        else:
+            host_in = {s: t.detach().to("cpu").pin_memory() for s, t in src.items()}
+            host_out = {s: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for s, t in src.items()}
+
+            def e2e_step():
+                for s in work:
+                    work[s].copy_(host_in[s], non_blocking=True)
+                    mo.muon_orthogonalize(work[s], steps=5, mode=args.form)
+                    host_out[s].copy_(work[s], non_blocking=True)
+            h2d = bytes_in
+            d2h = bytes_in
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world, dev)
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / e2e_steps
+        e2e = {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
+               "note": "pinned host grads -> HBM, muon_step, params -> pinned host, per step"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample = cpu_oracle_step_ms(w, args.cpu_seconds, args.form)
+        cpu = {"value": round(v, 2), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": round(ms_per_step, 4), "unit": "ms",
+            "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+            "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; shapes of the named model family, random values)",
+            "config": {"workload": w.name, "workload_id": w.wid, "matrices": w.count,
+                       "elements": w.elements, "ns_steps": 5, "ns_form": args.form,
+                       "coeffs": [3.4445, -4.775, 2.0315], "momentum": 0.95, "nesterov": True,
+                       "lr": 6e-4, "momentum_dtype": w.momentum_dtype, "param_dtype": w.param_dtype,
+                       "l2": f"inputs larger than L2: {in_bytes_resident / 1e6:.0f} MB read per step",
+                       "parallelism": f"replica x{world} (independent per GPU)"},
+            "ns_tflops_per_step": round(ns_tflops, 2),
+            "roofline": roofline, "roofline_momentum": roofline_mom,
+            "gpu_launches": int(launches),
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    budget = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_step_ms(w, budget, args.form)
+    vals = []
+    cores, sample = None, None
+    for _ in range(args.steps):
+        v, cores, sample = cpu_oracle_step_ms(w, budget, args.form)
+        vals.append(v)
+    value = statistics.fmean(vals)
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "ms",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(value, 2), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": w.name, "workload_id": w.wid, "matrices": w.count,
+                   "elements": w.elements, "ns_steps": 5, "ns_form": args.form},
+        "cpu_baseline": {"value": round(value, 2), "unit": "ms", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "ms", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,174 @@
+/*
+ * muon.h -- C ABI of the B200 (sm_100a) Muon optimizer-step library.
+ *
+ * The library orthogonalises 2D momentum matrices with Newton-Schulz (NS)
+ * iterations and applies the Muon update, entirely in CUDA kernels on the
+ * bound stream.  Sources of the method (web pages, cited by title + section):
+ *
+ *  [Gram-NS]       "GPU เร่งความเร็วใหม่! อัลกอริทึม Gram Newton-Schulz ..."
+ *                  (itsolotime.com): Muon = steepest descent under the spectral
+ *                  norm with polar(X) = U V^T approximated by NS, three matrix
+ *                  products per standard step ("ข้อได้เปรียบของอัลกอริทึม");
+ *                  the Gram form iterates on R = X X^T via p(t) = t q(t^2) and
+ *                  needs a restart in half precision
+ *                  ("ความท้าทายด้านความเสถียรและแนวทางแก้ไข").
+ *  [NanoGPT-Muon]  "2 分钟训练 124M 参数 NanoGPT：Muon 优化器与工程复现实践"
+ *                  (blog.hotdry.top): coefficients (3.4445, -4.7750, 2.0315),
+ *                  five steps, bfloat16 ("Newton-Schulz 迭代的系数调优与 FLOP
+ *                  开销分析"); momentum 0.95 with Nesterov ("工程复现清单").
+ *
+ * Conventions common to every call
+ *  - Matrices are dense row-major, rows x cols, element (i, j) at i*cols + j.
+ *  - The iteration runs on the short side: a matrix with rows > cols is
+ *    processed as its transpose and the result is written back in the
+ *    caller's layout.
+ *  - All tensor pointers are DEVICE pointers owned by the caller; arrays of
+ *    pointers, shapes and coefficients are HOST arrays read during the call.
+ *  - Work is enqueued asynchronously on the stream set by muon_set_stream
+ *    (default: the legacy default stream).  No call synchronises the host
+ *    except muon_device_status and muon_profile_read.
+ *  - The library owns a cached device workspace sized for the last shape set
+ *    (released by muon_release_workspace or at unload).  Calls are not
+ *    thread-safe; use one thread per library instance.
+ *  - Every call returns a status (< 0 on error) and never throws.  On an
+ *    argument error nothing is enqueued; muon_last_error() describes it.
+ */
+#ifndef MUON_B200_H
+#define MUON_B200_H
+
+#if defined(__GNUC__)
+#define MUON_API __attribute__((visibility("default")))
+#else
+#define MUON_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MUON_VERSION 10000 /* 1.0.0 */
+
+/* status codes */
+#define MUON_OK 0
+#define MUON_ERR_INVALID_ARG (-1) /* null pointer, non-positive size, bad steps/count */
+#define MUON_ERR_UNSUPPORTED (-2) /* dtype / mode combination not provided */
+#define MUON_ERR_CUDA (-3)        /* a CUDA runtime or driver call failed */
+#define MUON_ERR_NO_MEMORY (-4)   /* workspace allocation failed */
+#define MUON_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out */
+#define MUON_ERR_NONFINITE (-6)   /* ||U||_F was not finite for some matrix */
+
+/* mode bits of muon_orthogonalize and muon_config.mode */
+#define MUON_NS_STANDARD 0  /* A = X X^T, B = bA + cA^2, X <- aX + BX          */
+#define MUON_NS_GRAM 1      /* iterate on R = X X^T with restarts, O = Q X       */
+#define MUON_NS_AUTO 2      /* per matrix: Gram iff its FLOP count is lower      */
+#define MUON_NS_FORM_MASK 0xff
+#define MUON_PREC_FP32 0x100 /* fp32 check path: X is fp32, all math fp32 SIMT */
+
+/* element types */
+#define MUON_DTYPE_BF16 0
+#define MUON_DTYPE_F32 1
+
+#define MUON_MAX_STEPS 16
+
+typedef struct muon_config {
+    int steps;                        /* NS steps T for muon_step, 0..MUON_MAX_STEPS (default 5) */
+    float coeffs[3 * MUON_MAX_STEPS]; /* (a, b, c) of step k at [3k..3k+2] (default tuned set)  */
+    int mode;                         /* NS form for muon_step (default MUON_NS_AUTO)           */
+    unsigned restart_mask;            /* Gram form: bit k (k >= 1) restarts before step k;
+                                         used by both entry points (default 1u << 2)            */
+    float eps;                        /* added to the Frobenius norm (default 1e-7)             */
+    int momentum_dtype;               /* MUON_DTYPE_BF16 (default) or MUON_DTYPE_F32            */
+    int param_dtype;                  /* MUON_DTYPE_F32 (default) or MUON_DTYPE_BF16            */
+} muon_config;
+
+/* Library version (MUON_VERSION of the build). */
+MUON_API int muon_version(void);
+
+/* Fill *cfg with the defaults listed above.  Returns MUON_ERR_INVALID_ARG if cfg is NULL. */
+MUON_API int muon_default_config(muon_config* cfg);
+
+/* Validate and install *cfg for subsequent calls (copied). */
+MUON_API int muon_set_config(const muon_config* cfg);
+
+/* Copy the installed config into *cfg. */
+MUON_API int muon_get_config(muon_config* cfg);
+
+/* Bind the cudaStream_t (passed as void*) that all later work is enqueued on. NULL = default stream. */
+MUON_API int muon_set_stream(void* stream);
+
+/* Human-readable description of the last error of this thread ("" if none). */
+MUON_API const char* muon_last_error(void);
+
+/* Free the cached workspace and plans (waits for the bound stream first). */
+MUON_API int muon_release_workspace(void);
+
+/*
+ * Synchronise the bound stream, then read and clear the device status word.
+ * Returns MUON_OK, MUON_ERR_TIMEOUT (a kernel's bounded wait ran out; its
+ * outputs are undefined) or MUON_ERR_NONFINITE (a matrix had a non-finite
+ * Frobenius norm; that matrix's outputs were left untouched).  If bad_index
+ * is not NULL it receives the index of the first non-finite matrix (or -1).
+ */
+MUON_API int muon_device_status(int* bad_index);
+
+/*
+ * muon_orthogonalize -- X <- NS_T(X / (||X||_F + eps)) for a batch of matrices.
+ *   [Gram-NS] "ข้อได้เปรียบของอัลกอริทึม" (polar via NS, standard and Gram forms);
+ *   [NanoGPT-Muon] "Newton-Schulz 迭代的系数调优" (coefficients, T = 5).
+ * batch   number of matrices (>= 1), stored back to back in X
+ * m, n    rows and columns of each matrix (>= 1); the iteration uses the
+ *         shorter side (Gram matrix min(m,n) x min(m,n))
+ * X       device pointer, in place; bf16 by default, fp32 with MUON_PREC_FP32.
+ *         bf16 X must be 16-byte aligned when n % 8 == 0 (any alignment
+ *         otherwise: a padded internal copy is used)
+ * coeffs  host array of 3*steps floats, (a, b, c) of step k at [3k..3k+2]
+ * steps   T in 0..MUON_MAX_STEPS; 0 returns the normalised X
+ * mode    MUON_NS_STANDARD | MUON_NS_GRAM | MUON_NS_AUTO, optionally | MUON_PREC_FP32
+ * eps and the Gram restart schedule come from the installed config.
+ * A zero matrix returns zeros.
+ */
+MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* coeffs, int steps, int mode);
+
+/*
+ * muon_step -- one Muon step over count 2D parameters.
+ *   [NanoGPT-Muon] "从 SGD 到 Muon", "工程复现清单"; [Gram-NS] "ข้อได้เปรียบของอัลกอริทึม":
+ *     M <- mu*M + G;  U = G + mu*M (nesterov) or U = M;
+ *     O = NS_T(U / (||U||_F + eps));  W <- W - lr*O.
+ * params      host array of count device pointers, param_dtype, updated in place
+ * grads       host array of count device pointers, bf16, read only
+ * momentum    host array of count device pointers, momentum_dtype, updated in place
+ * shape_list  host int[2*count]: rows_i, cols_i of parameter i (>= 1)
+ * Coefficients, steps, NS form, restarts, eps and dtypes come from the
+ * installed config.  Pointers must be 16-byte aligned for the vectorised
+ * path (otherwise a scalar path is used).  Distinct parameters must not
+ * overlap.
+ */
+MUON_API int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
+              float lr, const int* shape_list, int count);
+
+/* ---- tracing ------------------------------------------------------------ */
+
+typedef struct muon_kernel_stats {
+    char name[32];    /* kernel kind: "momentum_norm", "gemm_tc", "gemm_f32", "scale_apply" */
+    long long launches;
+    double total_ms;  /* sum of CUDA-event durations on the launching stream */
+    double flops;     /* algorithmic FLOPs summed over launches (symmetric products at half cost) */
+    double bytes;     /* algorithmic HBM bytes summed over launches */
+} muon_kernel_stats;
+
+/* When on, a CUDA event pair is recorded on the bound stream around every launch. */
+MUON_API int muon_profile_enable(int on);
+
+/* Synchronise, fold pending events, copy up to max entries; *count receives the number of kinds. */
+MUON_API int muon_profile_read(muon_kernel_stats* out, int max, int* count);
+
+/* Clear the accumulated statistics. */
+MUON_API int muon_profile_reset(void);
+
+/* Number of kernels this library has launched since load. */
+MUON_API long long muon_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MUON_B200_H */

@@ -1,0 +1,166 @@
+// Element access and the fused GEMM epilogue shared by the tensor-core and
+// the fp32 SIMT kernels.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "muon_internal.h"
+
+namespace muon {
+
+__device__ __forceinline__ float ld_elem(const void* p, int dt, long long i) {
+    if (dt == DT_F32) return static_cast<const float*>(p)[i];
+    if (dt == DT_BF16) return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+    return __half2float(static_cast<const __half*>(p)[i]);
+}
+
+__device__ __forceinline__ void st_elem(void* p, int dt, long long i, float v) {
+    if (dt == DT_F32) {
+        static_cast<float*>(p)[i] = v;
+    } else if (dt == DT_BF16) {
+        static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(v);
+    } else {
+        static_cast<__half*>(p)[i] = __float2half_rn(v);
+    }
+}
+
+// Unpack 8 16-bit values held in a uint4.
+__device__ __forceinline__ void unpack8(const uint4& q, int dt, float* out) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (dt == DT_BF16) {
+            __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
+            float2 f = __bfloat1622float2(h);
+            out[2 * i] = f.x;
+            out[2 * i + 1] = f.y;
+        } else {
+            __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
+            float2 f = __half22float2(h);
+            out[2 * i] = f.x;
+            out[2 * i + 1] = f.y;
+        }
+    }
+}
+
+__device__ __forceinline__ uint4 pack8(const float* v, int dt) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (dt == DT_BF16) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        } else {
+            __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+            w[i] = *reinterpret_cast<uint32_t*>(&h);
+        }
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Load 32 consecutive elements of one row (columns col0 .. col0+31); columns
+// at or beyond col0 + nvalid read as 0.
+__device__ __forceinline__ void load_row32(const void* base, int dt, long long ld, long long row, int col0,
+                                           int nvalid, float* out) {
+    const long long off = row * ld + col0;
+    if (dt != DT_F32 && nvalid == 32 && ((reinterpret_cast<uintptr_t>(base) + off * 2) & 15) == 0) {
+        const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) unpack8(p[q], dt, out + 8 * q);
+        return;
+    }
+    if (dt == DT_F32 && nvalid == 32 && ((reinterpret_cast<uintptr_t>(base) + off * 4) & 15) == 0) {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float4 f = p[q];
+            out[4 * q] = f.x;
+            out[4 * q + 1] = f.y;
+            out[4 * q + 2] = f.z;
+            out[4 * q + 3] = f.w;
+        }
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) out[j] = (j < nvalid) ? ld_elem(base, dt, off + j) : 0.f;
+}
+
+// Store columns [jmin, nvalid) of a 32-wide row segment.
+__device__ __forceinline__ void store_row32(void* base, int dt, long long ld, long long row, int col0, int jmin,
+                                            int nvalid, const float* v) {
+    const long long off = row * ld + col0;
+    if (jmin == 0 && nvalid == 32) {
+        if (dt != DT_F32 && ((reinterpret_cast<uintptr_t>(base) + off * 2) & 15) == 0) {
+            uint4* p = reinterpret_cast<uint4*>(static_cast<uint16_t*>(base) + off);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) p[q] = pack8(v + 8 * q, dt);
+            return;
+        }
+        if (dt == DT_F32 && ((reinterpret_cast<uintptr_t>(base) + off * 4) & 15) == 0) {
+            float4* p = reinterpret_cast<float4*>(static_cast<float*>(base) + off);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) p[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            return;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        if (j >= jmin && j < nvalid) st_elem(base, dt, off + j, v[j]);
+}
+
+// Apply the fused epilogue to a 32-column row segment of the accumulator:
+// row `row`, columns col0 .. col0 + 31 of an M x N output.  `sig` is the
+// problem's sigma (already loaded).
+__device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, int M, int N, long long row, int col0,
+                                               float* acc) {
+    if (row >= M) return;
+    const int nvalid = min(32, N - col0);
+    if (nvalid <= 0) return;
+    // symmetric outputs: only columns >= row are produced here
+    const int jmin = ep.sym ? max(0, static_cast<int>(row - col0)) : 0;
+    if (jmin >= nvalid) return;
+    float t1[32];
+    if (ep.c1) {
+        load_row32(ep.c1, ep.c1_dt, ep.ldc1, row, col0, nvalid, t1);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = fmaf(ep.beta, t1[j], ep.alpha * acc[j]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = ep.alpha * acc[j];
+    }
+    if (sig == 0.f) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+    } else if (sig != 1.f) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] *= sig;
+    }
+    if (ep.c2) {
+        load_row32(ep.c2, ep.c2_dt, ep.ldc2, row, col0, nvalid, t1);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[j] = fmaf(ep.gamma, t1[j], acc[j]);
+    }
+    if (ep.delta != 0.f) {
+        const long long d = row - col0;
+        if (d >= 0 && d < 32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j == d) acc[j] += ep.delta;
+        }
+    }
+    store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, jmin, nvalid, acc);
+    if (ep.o2) store_row32(ep.o2, ep.o2_dt, ep.ldo2, row, col0, jmin, nvalid, acc);
+    if (ep.sym) {
+        // mirrored copy of the strictly-upper part: (col, row)
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const long long col = col0 + j;
+            if (j < nvalid && col > row) {
+                st_elem(ep.o1, ep.o1_dt, col * ep.ldo1 + row, acc[j]);
+                if (ep.o2) st_elem(ep.o2, ep.o2_dt, col * ep.ldo2 + row, acc[j]);
+            }
+        }
+    }
+}
+
+}  // namespace muon

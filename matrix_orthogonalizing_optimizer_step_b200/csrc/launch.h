@@ -1,0 +1,65 @@
+// Internal launch interface between the planner and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "muon_internal.h"
+
+namespace muon {
+
+struct TcLaunch {
+    const TcProblem* problems;
+    const uint2* tiles;  // {problem index, (tile_row << 16) | tile_col}
+    int ntiles;
+    const CUtensorMap* maps;
+    const int* bad;       // per-matrix non-finite flags
+    DeviceStatus* status;
+};
+
+size_t gemm_tc_smem_bytes();
+int gemm_tc_tile_m();
+int gemm_tc_tile_n();
+cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream);
+
+struct F32Launch {
+    const F32Problem* problems;
+    int nproblems;
+    int max_m, max_n;
+    const int* bad;
+};
+cudaError_t launch_gemm_f32(const F32Launch& L, cudaStream_t stream);
+
+struct MomLaunch {
+    const MomMatrix* mats;
+    int nmats;
+    long long nchunks;
+    int in_dt;    // dtype of g (bf16 or f32)
+    int mom_dt;   // dtype of m (bf16 or f32), ignored without momentum
+    int u_dt;     // dtype of the workspace copy (bf16 or f32)
+    int has_momentum;
+    int nesterov;
+    float mu;
+    float lr;           // learning rate of a Muon step (0 for orthogonalize)
+    double eps;
+    float* partials;    // one per chunk
+    int* counters;      // one per matrix, zero between launches
+    float* scale;       // per matrix i: [4i] = s, [4i+1] = s*s, [4i+2] = -lr*s, [4i+3] = -lr
+    int* bad;           // per matrix non-finite flag
+    DeviceStatus* status;
+    int mat_index_base; // index of mats[0] in the caller's numbering (status reporting)
+};
+cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream);
+
+struct ScaleLaunch {
+    const ScaleMatrix* mats;
+    int nmats;
+    long long nchunks;
+    int u_dt, out_dt;
+    int update;  // 0: out = s*U;  1: out -= lr*s*U
+    float lr;
+    const float* scale;
+    const int* bad;
+};
+cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream);
+
+}  // namespace muon

@@ -1,0 +1,360 @@
+// C ABI of the Muon library (include/muon.h): argument validation, config,
+// stream binding, the device status word, tracing, and the two entry points.
+// No exception crosses this boundary; every entry point returns a status.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <deque>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "plan.h"
+
+using namespace muon;
+
+namespace {
+
+thread_local std::string g_err;
+muon_config g_cfg;
+bool g_cfg_init = false;
+cudaStream_t g_stream = nullptr;
+std::atomic<long long> g_launches{0};
+
+struct DeviceState {
+    int device = -1;
+    int num_sms = 0;
+    int cc_major = 0, cc_minor = 0;
+    DeviceStatus* status = nullptr;
+    std::unique_ptr<Plan> plan;
+};
+std::deque<DeviceState> g_devs;  // deque: references stay valid on growth
+
+int fail(int code, const std::string& msg) {
+    g_err = msg;
+    return code;
+}
+
+// Defaults: five steps of the tuned quintic (3.4445, -4.7750, 2.0315)
+// ([NanoGPT-Muon] "Newton-Schulz 迭代的系数调优"), per-matrix choice of the
+// cheaper form, one Gram restart before step 2, eps 1e-7, bf16 momentum,
+// fp32 parameters.
+void fill_defaults(muon_config* c) {
+    std::memset(c, 0, sizeof(*c));
+    c->steps = 5;
+    for (int k = 0; k < MUON_MAX_STEPS; ++k) {
+        c->coeffs[3 * k] = 3.4445f;
+        c->coeffs[3 * k + 1] = -4.7750f;
+        c->coeffs[3 * k + 2] = 2.0315f;
+    }
+    c->mode = MUON_NS_AUTO;
+    c->restart_mask = 1u << 2;
+    c->eps = 1e-7f;
+    c->momentum_dtype = MUON_DTYPE_BF16;
+    c->param_dtype = MUON_DTYPE_F32;
+}
+
+void ensure_cfg() {
+    if (g_cfg_init) return;
+    fill_defaults(&g_cfg);
+    g_cfg_init = true;
+}
+
+int check_cfg(const muon_config& c) {
+    if (c.steps < 0 || c.steps > MUON_MAX_STEPS) return fail(MUON_ERR_INVALID_ARG, "config.steps out of range");
+    if ((c.mode & ~MUON_NS_FORM_MASK) != 0 || c.mode < 0 || c.mode > MUON_NS_AUTO)
+        return fail(MUON_ERR_INVALID_ARG, "config.mode must be MUON_NS_STANDARD, MUON_NS_GRAM or MUON_NS_AUTO");
+    if (!(c.eps >= 0.f) || !std::isfinite(c.eps)) return fail(MUON_ERR_INVALID_ARG, "config.eps must be finite and >= 0");
+    for (int i = 0; i < 3 * c.steps; ++i)
+        if (!std::isfinite(c.coeffs[i])) return fail(MUON_ERR_INVALID_ARG, "config.coeffs must be finite");
+    if (c.momentum_dtype != MUON_DTYPE_BF16 && c.momentum_dtype != MUON_DTYPE_F32)
+        return fail(MUON_ERR_UNSUPPORTED, "config.momentum_dtype must be BF16 or F32");
+    if (c.param_dtype != MUON_DTYPE_BF16 && c.param_dtype != MUON_DTYPE_F32)
+        return fail(MUON_ERR_UNSUPPORTED, "config.param_dtype must be BF16 or F32");
+    return MUON_OK;
+}
+
+// Current device's state; allocates the status word on first use.
+int device_state(DeviceState** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MUON_ERR_CUDA, std::string("no CUDA device: ") + cudaGetErrorString(e));
+    }
+    for (DeviceState& d : g_devs)
+        if (d.device == dev) {
+            *out = &d;
+            return MUON_OK;
+        }
+    DeviceState d;
+    d.device = dev;
+    cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (cudaMalloc(&d.status, sizeof(DeviceStatus)) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MUON_ERR_NO_MEMORY, "status word allocation failed");
+    }
+    const DeviceStatus init{0, 0x7fffffff};
+    cudaMemcpy(d.status, &init, sizeof(init), cudaMemcpyHostToDevice);
+    d.plan.reset(new Plan());
+    g_devs.push_back(std::move(d));
+    *out = &g_devs.back();
+    return MUON_OK;
+}
+
+// ---- tracing ------------------------------------------------------------------
+
+struct Pending {
+    cudaEvent_t a, b;
+    int kind;
+    double flops, bytes;
+};
+
+struct Profiler : ProfileSink {
+    bool on = false;
+    std::vector<Pending> pending;
+    std::vector<cudaEvent_t> pool;
+    muon_kernel_stats stats[4];
+    cudaEvent_t cur = nullptr;
+    Profiler() { reset(); }
+    void reset() {
+        static const char* names[4] = {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply"};
+        for (int i = 0; i < 4; ++i) {
+            std::memset(&stats[i], 0, sizeof(stats[i]));
+            std::strncpy(stats[i].name, names[i], sizeof(stats[i].name) - 1);
+        }
+    }
+    cudaEvent_t get() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e;
+        cudaEventCreate(&e);
+        return e;
+    }
+    void before(cudaStream_t s) override {
+        cur = get();
+        cudaEventRecord(cur, s);
+    }
+    void after(cudaStream_t s, int kind, double flops, double bytes) override {
+        cudaEvent_t b = get();
+        cudaEventRecord(b, s);
+        // LaunchRec kinds: MOM, TC, F32, SCALE -> stats slots 0..3
+        pending.push_back({cur, b, kind, flops, bytes});
+        cur = nullptr;
+    }
+    void fold() {
+        for (Pending& p : pending) {
+            float ms = 0.f;
+            cudaEventSynchronize(p.b);
+            cudaEventElapsedTime(&ms, p.a, p.b);
+            muon_kernel_stats& st = stats[p.kind];
+            st.launches += 1;
+            st.total_ms += ms;
+            st.flops += p.flops;
+            st.bytes += p.bytes;
+            pool.push_back(p.a);
+            pool.push_back(p.b);
+        }
+        pending.clear();
+    }
+};
+Profiler g_prof;
+
+int run_plan(DeviceState* ds, const PlanRequest& rq) {
+    std::string err;
+    Plan& plan = *ds->plan;
+    if (!plan.same_shape_key(rq)) {
+        // tables of the previous plan may still be read by queued kernels
+        cudaError_t e = cudaStreamSynchronize(g_stream);
+        if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("stream sync failed: ") + cudaGetErrorString(e));
+        const int st = plan.build(rq, ds->status, ds->num_sms, g_stream, err);
+        if (st != MUON_OK) {
+            plan.release();
+            return fail(st, err);
+        }
+    }
+    plan.set_scalars(rq.mu, rq.nesterov, rq.lr);
+    long long launched = 0;
+    const int st = plan.run(g_stream, g_prof.on ? &g_prof : nullptr, &launched, err);
+    g_launches += launched;
+    if (st != MUON_OK) return fail(st, err);
+    return MUON_OK;
+}
+
+int check_device(DeviceState** ds, bool need_tc) {
+    const int st = device_state(ds);
+    if (st != MUON_OK) return st;
+    if (need_tc && (*ds)->cc_major != 10)
+        return fail(MUON_ERR_UNSUPPORTED, "the tensor-core path needs an sm_100 GPU (B200)");
+    return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int muon_version(void) { return MUON_VERSION; }
+
+int muon_default_config(muon_config* cfg) {
+    if (!cfg) return fail(MUON_ERR_INVALID_ARG, "cfg is NULL");
+    fill_defaults(cfg);
+    return MUON_OK;
+}
+
+int muon_set_config(const muon_config* cfg) {
+    if (!cfg) return fail(MUON_ERR_INVALID_ARG, "cfg is NULL");
+    const int st = check_cfg(*cfg);
+    if (st != MUON_OK) return st;
+    ensure_cfg();
+    g_cfg = *cfg;
+    return MUON_OK;
+}
+
+int muon_get_config(muon_config* cfg) {
+    if (!cfg) return fail(MUON_ERR_INVALID_ARG, "cfg is NULL");
+    ensure_cfg();
+    *cfg = g_cfg;
+    return MUON_OK;
+}
+
+int muon_set_stream(void* stream) {
+    g_stream = static_cast<cudaStream_t>(stream);
+    return MUON_OK;
+}
+
+const char* muon_last_error(void) { return g_err.c_str(); }
+
+int muon_release_workspace(void) {
+    cudaStreamSynchronize(g_stream);
+    for (DeviceState& d : g_devs)
+        if (d.plan) d.plan->release();
+    return MUON_OK;
+}
+
+int muon_device_status(int* bad_index) {
+    if (bad_index) *bad_index = -1;
+    DeviceState* ds = nullptr;
+    int st = device_state(&ds);
+    if (st != MUON_OK) return st;
+    cudaError_t e = cudaStreamSynchronize(g_stream);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("stream sync failed: ") + cudaGetErrorString(e));
+    DeviceStatus h;
+    e = cudaMemcpy(&h, ds->status, sizeof(h), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("status read failed: ") + cudaGetErrorString(e));
+    const DeviceStatus init{0, 0x7fffffff};
+    cudaMemcpy(ds->status, &init, sizeof(init), cudaMemcpyHostToDevice);
+    if (bad_index && h.first_bad != 0x7fffffff) *bad_index = h.first_bad;
+    if (h.bits & ST_TIMEOUT) return fail(MUON_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+    if (h.bits & ST_NONFINITE) return fail(MUON_ERR_NONFINITE, "non-finite Frobenius norm");
+    return MUON_OK;
+}
+
+int muon_orthogonalize(int batch, int m, int n, void* X, const float* coeffs, int steps, int mode) {
+    ensure_cfg();
+    if (batch < 1 || m < 1 || n < 1) return fail(MUON_ERR_INVALID_ARG, "batch, m and n must be >= 1");
+    if (!X) return fail(MUON_ERR_INVALID_ARG, "X is NULL");
+    if (steps < 0 || steps > MUON_MAX_STEPS) return fail(MUON_ERR_INVALID_ARG, "steps out of range");
+    if (steps > 0 && !coeffs) return fail(MUON_ERR_INVALID_ARG, "coeffs is NULL");
+    const int form = mode & MUON_NS_FORM_MASK;
+    const bool fp32 = (mode & MUON_PREC_FP32) != 0;
+    if ((mode & ~(MUON_NS_FORM_MASK | MUON_PREC_FP32)) != 0 || form > MUON_NS_AUTO)
+        return fail(MUON_ERR_INVALID_ARG, "unknown mode bits");
+    for (int i = 0; i < 3 * steps; ++i)
+        if (!std::isfinite(coeffs[i])) return fail(MUON_ERR_INVALID_ARG, "coeffs must be finite");
+    if (static_cast<long long>(m) > (1LL << 30) || static_cast<long long>(n) > (1LL << 30))
+        return fail(MUON_ERR_INVALID_ARG, "dimension too large");
+    DeviceState* ds = nullptr;
+    int st = check_device(&ds, !fp32);
+    if (st != MUON_OK) return st;
+
+    PlanRequest rq;
+    const int es = fp32 ? 4 : 2;
+    for (int b = 0; b < batch; ++b) {
+        char* p = static_cast<char*>(X) + static_cast<size_t>(b) * m * n * es;
+        rq.rows.push_back(m);
+        rq.cols.push_back(n);
+        rq.in.push_back(p);
+        rq.out.push_back(p);
+    }
+    rq.in_dt = fp32 ? DT_F32 : DT_BF16;
+    rq.out_dt = rq.in_dt;
+    rq.is_step = false;
+    rq.fp32_path = fp32;
+    rq.form = form;
+    rq.steps = steps;
+    rq.coeffs.assign(coeffs ? coeffs : nullptr, coeffs ? coeffs + 3 * steps : nullptr);
+    rq.restart_mask = g_cfg.restart_mask;
+    rq.eps = g_cfg.eps;
+    rq.device = ds->device;
+    return run_plan(ds, rq);
+}
+
+int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov, float lr,
+              const int* shape_list, int count) {
+    ensure_cfg();
+    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
+    if (!params || !grads || !momentum || !shape_list)
+        return fail(MUON_ERR_INVALID_ARG, "params, grads, momentum and shape_list must not be NULL");
+    if (!std::isfinite(mu) || !std::isfinite(lr)) return fail(MUON_ERR_INVALID_ARG, "mu and lr must be finite");
+    PlanRequest rq;
+    for (int i = 0; i < count; ++i) {
+        const int r = shape_list[2 * i], c = shape_list[2 * i + 1];
+        if (r < 1 || c < 1) return fail(MUON_ERR_INVALID_ARG, "shape_list entries must be >= 1");
+        if (!params[i] || !grads[i] || !momentum[i])
+            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/momentum");
+        rq.rows.push_back(r);
+        rq.cols.push_back(c);
+        rq.in.push_back(grads[i]);
+        rq.mom.push_back(momentum[i]);
+        rq.out.push_back(params[i]);
+    }
+    DeviceState* ds = nullptr;
+    int st = check_device(&ds, true);
+    if (st != MUON_OK) return st;
+    rq.in_dt = DT_BF16;
+    rq.mom_dt = g_cfg.momentum_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
+    rq.out_dt = g_cfg.param_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
+    rq.is_step = true;
+    rq.fp32_path = false;
+    rq.form = g_cfg.mode;
+    rq.steps = g_cfg.steps;
+    rq.coeffs.assign(g_cfg.coeffs, g_cfg.coeffs + 3 * g_cfg.steps);
+    rq.restart_mask = g_cfg.restart_mask;
+    rq.eps = g_cfg.eps;
+    rq.mu = mu;
+    rq.nesterov = nesterov ? 1 : 0;
+    rq.lr = lr;
+    rq.device = ds->device;
+    return run_plan(ds, rq);
+}
+
+int muon_profile_enable(int on) {
+    g_prof.on = on != 0;
+    return MUON_OK;
+}
+
+int muon_profile_read(muon_kernel_stats* out, int max, int* count) {
+    g_prof.fold();
+    if (count) *count = 4;
+    if (out)
+        for (int i = 0; i < max && i < 4; ++i) out[i] = g_prof.stats[i];
+    return MUON_OK;
+}
+
+int muon_profile_reset(void) {
+    g_prof.fold();
+    g_prof.reset();
+    return MUON_OK;
+}
+
+long long muon_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

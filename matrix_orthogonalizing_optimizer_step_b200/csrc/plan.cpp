@@ -1,0 +1,793 @@
+// Planner: groups matrices by shape, lays out the workspace, writes the
+// Newton-Schulz op chain of every group and lowers the chains into grouped
+// kernel launches.  See plan.h.
+//
+// Newton-Schulz forms ([Gram-NS] "ข้อได้เปรียบของอัลกอริทึม" and
+// "ความท้าทายด้านความเสถียรและแนวทางแก้ไข"; coefficients from [NanoGPT-Muon]
+// "Newton-Schulz 迭代的系数调优"), for X (n x m, n <= m) with X0 = s U,
+// s = 1 / (||U||_F + eps):
+//
+//   standard, per step k:   A = X X^T ;  B = b A + c A^2 ;  X <- a X + B X
+//   Gram, per step k:       Z = a I + b R + c R^2 ;  Q <- Z Q ;  R <- Z (Z R)
+//                           (R = X X^T at the start of every segment; a restart
+//                           before step k sets X <- Q X, R <- X X^T, Q <- I;
+//                           the result is Q X)
+//
+// Precision of the tensor-core path: X, A, B and the bf16 copy of Q used in
+// Q X are bf16; the Gram quantities R, Z, Z R, Q are fp16 (the Gram form is
+// run in half precision with restarts, as the Gram page describes); every
+// product accumulates in fp32 and every stored matrix is rounded once.
+#include "plan.h"
+
+#include <algorithm>
+#include <cstring>
+#include <map>
+#include <tuple>
+
+#include "../../include/muon.h"
+
+namespace muon {
+namespace {
+
+enum Buf { X0 = 0, X1, X2, BA, BB, BR, BZ0, BZ1, BZR, BQ0, BQ1, BQBF, NBUF };
+constexpr int OUTB = 100;  // the caller's output / parameter, in the caller's layout
+enum OpKind { OP_SYRK, OP_PROD, OP_APPLY };
+enum SigmaKind { SIG_NONE = 0, SIG_S = 1, SIG_S2 = 2 };
+
+struct OpDesc {
+    int kind = OP_PROD;
+    int a = -1, b = -1;  // SYRK: a = b = X; PROD: n x n factors; APPLY: a = n x n factor, b = X
+    float alpha = 1.f, beta = 0.f, gamma = 0.f, delta = 0.f;
+    int sigma = SIG_NONE;
+    int c1 = -1, c2 = -1, o1 = -1, o2 = -1;
+    bool sym = false;
+    bool final = false;
+};
+using Slot = std::vector<OpDesc>;
+
+struct Group {
+    int n = 0, m = 0;
+    bool trans = false;
+    int form = FORM_STANDARD;
+    std::vector<int> mats;
+    long long rows_w = 0, cols_w = 0;  // X buffers in the caller's layout
+    long long ldx = 0, ldn = 0;
+    bool used[NBUF] = {};
+    int dt[NBUF] = {};
+    size_t off[NBUF] = {};
+    long long bstride[NBUF] = {};  // bytes between consecutive matrices
+    std::vector<Slot> slots;
+};
+
+long long round_up(long long v, long long a) { return (v + a - 1) / a * a; }
+
+bool restart_at(unsigned mask, int k) { return k > 0 && k < 32 && ((mask >> k) & 1u); }
+
+// ---- op chains ---------------------------------------------------------------
+
+void make_final(OpDesc& op, const PlanRequest& rq) {
+    op.final = true;
+    op.o1 = OUTB;
+    if (rq.is_step) {
+        // W <- W - lr * O : the -lr factor is folded into the per-matrix sigma
+        op.c2 = OUTB;
+        op.gamma = 1.f;
+    }
+}
+
+void chain_standard(Group& g, const PlanRequest& rq) {
+    const int T = rq.steps;
+    int xcur = X0;
+    const int xring[2] = {X1, X2};
+    int ring = 0;
+    for (int k = 0; k < T; ++k) {
+        const float a = rq.coeffs[3 * k], b = rq.coeffs[3 * k + 1], c = rq.coeffs[3 * k + 2];
+        OpDesc syrk;
+        syrk.kind = OP_SYRK;
+        syrk.a = syrk.b = xcur;
+        syrk.sym = true;
+        syrk.sigma = (k == 0) ? SIG_S2 : SIG_NONE;
+        syrk.o1 = BA;
+        OpDesc prod;
+        prod.kind = OP_PROD;
+        prod.a = prod.b = BA;
+        prod.sym = true;
+        prod.alpha = c;
+        prod.beta = b;
+        prod.c1 = BA;
+        prod.o1 = BB;
+        OpDesc app;
+        app.kind = OP_APPLY;
+        app.a = BB;
+        app.b = xcur;
+        app.alpha = 1.f;
+        app.beta = a;
+        app.c1 = xcur;
+        app.sigma = (k == 0) ? SIG_S : SIG_NONE;
+        if (k == T - 1) {
+            make_final(app, rq);
+        } else {
+            app.o1 = xring[ring];
+            ring ^= 1;
+            xcur = app.o1;
+        }
+        g.slots.push_back({syrk});
+        g.slots.push_back({prod});
+        g.slots.push_back({app});
+    }
+}
+
+void chain_gram(Group& g, const PlanRequest& rq) {
+    const int T = rq.steps;
+    int xcur = X0;
+    bool x_scaled = false;  // X0 still carries the factor s
+    const int xring[2] = {X1, X2};
+    int ring = 0;
+    {
+        OpDesc syrk;
+        syrk.kind = OP_SYRK;
+        syrk.a = syrk.b = xcur;
+        syrk.sym = true;
+        syrk.sigma = SIG_S2;
+        syrk.o1 = BR;
+        g.slots.push_back({syrk});
+    }
+    int qsrc = -1;  // buffer holding Q, -1 = identity (segment start)
+    for (int k = 0; k < T; ++k) {
+        const float a = rq.coeffs[3 * k], b = rq.coeffs[3 * k + 1], c = rq.coeffs[3 * k + 2];
+        if (restart_at(rq.restart_mask, k)) {
+            // X <- Q X, R <- X X^T, Q <- I
+            OpDesc app;
+            app.kind = OP_APPLY;
+            app.a = BQBF;
+            app.b = xcur;
+            app.sigma = x_scaled ? SIG_NONE : SIG_S;
+            app.o1 = xring[ring];
+            ring ^= 1;
+            g.slots.push_back({app});
+            xcur = app.o1;
+            x_scaled = true;
+            OpDesc syrk;
+            syrk.kind = OP_SYRK;
+            syrk.a = syrk.b = xcur;
+            syrk.sym = true;
+            syrk.o1 = BR;
+            g.slots.push_back({syrk});
+            qsrc = -1;
+        }
+        const bool first = (qsrc == -1);
+        const bool last = (k == T - 1) || restart_at(rq.restart_mask, k + 1);
+        const int zb = (k & 1) ? BZ1 : BZ0;
+        // Z = a I + b R + c R^2
+        OpDesc p1;
+        p1.kind = OP_PROD;
+        p1.a = p1.b = BR;
+        p1.sym = true;
+        p1.alpha = c;
+        p1.beta = b;
+        p1.c1 = BR;
+        p1.delta = a;
+        p1.o1 = (first && last) ? BQBF : zb;  // a one-step segment only needs Q = Z
+        g.slots.push_back({p1});
+        Slot s2;
+        int qnext = zb;  // at a segment start Q = Z (same buffer)
+        if (!first) {
+            // Q <- Z Q
+            OpDesc p4;
+            p4.kind = OP_PROD;
+            p4.a = zb;
+            p4.b = qsrc;
+            p4.sym = true;
+            p4.o1 = last ? BQBF : (qsrc == BQ0 ? BQ1 : BQ0);
+            s2.push_back(p4);
+            qnext = p4.o1;
+        }
+        if (!last) {
+            // Z R
+            OpDesc p2;
+            p2.kind = OP_PROD;
+            p2.a = zb;
+            p2.b = BR;
+            p2.sym = true;
+            p2.o1 = BZR;
+            s2.push_back(p2);
+        }
+        if (!s2.empty()) g.slots.push_back(s2);
+        if (!last) {
+            // R <- Z (Z R)
+            OpDesc p3;
+            p3.kind = OP_PROD;
+            p3.a = zb;
+            p3.b = BZR;
+            p3.sym = true;
+            p3.o1 = BR;
+            g.slots.push_back({p3});
+        }
+        qsrc = qnext;
+    }
+    OpDesc fin;
+    fin.kind = OP_APPLY;
+    fin.a = BQBF;
+    fin.b = xcur;
+    fin.sigma = x_scaled ? SIG_NONE : SIG_S;
+    make_final(fin, rq);
+    g.slots.push_back({fin});
+}
+
+void mark_used(Group& g) {
+    for (const Slot& s : g.slots)
+        for (const OpDesc& op : s)
+            for (int b : {op.a, op.b, op.c1, op.c2, op.o1, op.o2})
+                if (b >= 0 && b < NBUF) g.used[b] = true;
+    g.used[X0] = true;
+}
+
+bool is_x_buf(int b) { return b == X0 || b == X1 || b == X2; }
+
+struct OperandGeom {
+    int buf;
+    bool mn;
+};
+
+void op_geometry(const Group& g, const OpDesc& op, int& M, int& N, int& K, OperandGeom& A, OperandGeom& B) {
+    switch (op.kind) {
+        case OP_SYRK:
+            M = N = g.n;
+            K = g.m;
+            A = {op.a, g.trans};
+            B = {op.b, g.trans};
+            break;
+        case OP_PROD:
+            M = N = K = g.n;
+            A = {op.a, false};
+            B = {op.b, false};  // symmetric: rows of b are its columns
+            break;
+        default:  // OP_APPLY
+            if (!g.trans) {
+                M = g.n, N = g.m, K = g.n;
+                A = {op.a, false};
+                B = {op.b, true};
+            } else {
+                M = g.m, N = g.n, K = g.n;
+                A = {op.b, false};
+                B = {op.a, false};
+            }
+    }
+}
+
+double op_flops(const Group& g, const OpDesc& op) {
+    const double n = g.n, m = g.m;
+    switch (op.kind) {
+        case OP_SYRK: return n * n * m;       // symmetric output: half of 2 n^2 m
+        case OP_PROD: return n * n * n;       // symmetric output: half of 2 n^3
+        default: return 2.0 * n * n * m;
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder(std::string& err) {
+    static EncodeTiledFn fn = nullptr;
+    if (fn) return fn;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) {
+        err = "cuTensorMapEncodeTiled unavailable";
+        return nullptr;
+    }
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+    return fn;
+}
+
+}  // namespace
+
+double ns_flops(int n, int m, int steps, int form, unsigned restart_mask) {
+    const double N = n, M = m;
+    if (form == FORM_STANDARD) return steps * (3.0 * N * N * M + N * N * N);
+    std::vector<int> starts = {0};
+    for (int k = 1; k < steps; ++k)
+        if (restart_at(restart_mask, k)) starts.push_back(k);
+    double total = 0;
+    for (size_t i = 0; i < starts.size(); ++i) {
+        const int s = starts[i], e = (i + 1 < starts.size()) ? starts[i + 1] : steps;
+        total += 3.0 * N * N * M;
+        for (int k = s; k < e; ++k) {
+            total += N * N * N;
+            if (k > s) total += N * N * N;
+            if (k < e - 1) total += 2.0 * N * N * N;
+        }
+    }
+    return total;
+}
+
+int resolve_form(int n, int m, int steps, int form, unsigned restart_mask) {
+    if (form != FORM_AUTO) return form;
+    return ns_flops(n, m, steps, FORM_GRAM, restart_mask) < ns_flops(n, m, steps, FORM_STANDARD, restart_mask)
+               ? FORM_GRAM
+               : FORM_STANDARD;
+}
+
+static std::vector<long long> make_key(const PlanRequest& rq) {
+    // Everything the tables depend on; mu, nesterov and lr are patched per call.
+    std::vector<long long> k;
+    k.reserve(16 + rq.rows.size() * 5 + rq.coeffs.size());
+    k.push_back(rq.device);
+    k.push_back(rq.is_step);
+    k.push_back(rq.fp32_path);
+    k.push_back(rq.form);
+    k.push_back(rq.steps);
+    k.push_back(rq.restart_mask);
+    int eb;
+    std::memcpy(&eb, &rq.eps, sizeof(float));
+    k.push_back(eb);
+    k.push_back(rq.in_dt);
+    k.push_back(rq.mom_dt);
+    k.push_back(rq.out_dt);
+    for (float c : rq.coeffs) {
+        int bits;
+        std::memcpy(&bits, &c, 4);
+        k.push_back(bits);
+    }
+    for (size_t i = 0; i < rq.rows.size(); ++i) {
+        k.push_back(rq.rows[i]);
+        k.push_back(rq.cols[i]);
+        k.push_back(reinterpret_cast<long long>(rq.in[i]));
+        k.push_back(reinterpret_cast<long long>(rq.mom.empty() ? nullptr : rq.mom[i]));
+        k.push_back(reinterpret_cast<long long>(rq.out[i]));
+    }
+    return k;
+}
+
+bool Plan::same_shape_key(const PlanRequest& rq) const { return !key_.empty() && make_key(rq) == key_; }
+
+void Plan::set_scalars(float mu, int nesterov, float lr) {
+    for (LaunchRec& l : launches) {
+        if (l.kind == LaunchRec::MOM) {
+            l.mom.mu = mu;
+            l.mom.nesterov = nesterov;
+            l.mom.lr = lr;
+        } else if (l.kind == LaunchRec::SCALE) {
+            l.sc.lr = lr;
+        }
+    }
+}
+
+void Plan::release() {
+    if (arena_) cudaFree(arena_);
+    arena_ = nullptr;
+    arena_bytes = 0;
+    launches.clear();
+    key_.clear();
+}
+
+int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaStream_t stream, std::string& err) {
+    // ---- key -------------------------------------------------------------------
+    launches.clear();
+    key_.clear();
+    total_flops = 0;
+    const int nm = static_cast<int>(rq.rows.size());
+    const bool f32 = rq.fp32_path;
+    const int tile_m = gemm_tc_tile_m(), tile_n = gemm_tc_tile_n();
+
+    // ---- groups ----------------------------------------------------------------
+    std::vector<Group> groups;
+    std::map<std::tuple<int, int, int, int>, int> gindex;
+    std::vector<int> mat_group(nm), mat_z(nm);
+    for (int i = 0; i < nm; ++i) {
+        const int r = rq.rows[i], c = rq.cols[i];
+        const bool trans = r > c;
+        const int n = trans ? c : r, m = trans ? r : c;
+        const int form = rq.steps > 0 ? resolve_form(n, m, rq.steps, rq.form, rq.restart_mask) : FORM_STANDARD;
+        auto key = std::make_tuple(n, m, static_cast<int>(trans), form);
+        auto it = gindex.find(key);
+        int gi;
+        if (it == gindex.end()) {
+            gi = static_cast<int>(groups.size());
+            gindex[key] = gi;
+            Group g;
+            g.n = n;
+            g.m = m;
+            g.trans = trans;
+            g.form = form;
+            g.rows_w = r;
+            g.cols_w = c;
+            g.ldx = round_up(c, 8);
+            g.ldn = round_up(n, 8);
+            groups.push_back(g);
+        } else {
+            gi = it->second;
+        }
+        mat_group[i] = gi;
+        mat_z[i] = static_cast<int>(groups[gi].mats.size());
+        groups[gi].mats.push_back(i);
+    }
+    for (Group& g : groups) {
+        if (rq.steps > 0) {
+            if (g.form == FORM_GRAM)
+                chain_gram(g, rq);
+            else
+                chain_standard(g, rq);
+        }
+        mark_used(g);
+        for (int b = 0; b < NBUF; ++b) {
+            if (f32)
+                g.dt[b] = DT_F32;
+            else if (b == BR || b == BZ0 || b == BZ1 || b == BZR || b == BQ0 || b == BQ1)
+                g.dt[b] = DT_F16;
+            else
+                g.dt[b] = DT_BF16;
+        }
+    }
+
+    // ---- workspace layout --------------------------------------------------------
+    size_t cursor = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = cursor;
+        cursor = static_cast<size_t>(round_up(static_cast<long long>(cursor + bytes), 1024));
+        return o;
+    };
+    for (Group& g : groups) {
+        const long long cnt = static_cast<long long>(g.mats.size());
+        for (int b = 0; b < NBUF; ++b) {
+            if (!g.used[b]) continue;
+            const long long rows = is_x_buf(b) ? g.rows_w : g.n;
+            const long long ld = is_x_buf(b) ? g.ldx : g.ldn;
+            g.bstride[b] = rows * ld * dtype_size(g.dt[b]);
+            g.off[b] = take(static_cast<size_t>(g.bstride[b] * cnt));
+        }
+    }
+    // per-matrix chunks of the momentum / normalise kernel
+    std::vector<MomMatrix> moms(nm);
+    long long nchunks = 0;
+    for (int i = 0; i < nm; ++i) {
+        const long long numel = static_cast<long long>(rq.rows[i]) * rq.cols[i];
+        moms[i].chunk_begin = nchunks;
+        moms[i].nchunks = static_cast<int>((numel + kMomChunk - 1) / kMomChunk);
+        nchunks += moms[i].nchunks;
+    }
+    const size_t off_partials = take(sizeof(float) * nchunks);
+    const size_t off_counters = take(sizeof(int) * nm);
+    const size_t off_scale = take(sizeof(float) * 4 * nm);
+    const size_t off_bad = take(sizeof(int) * nm);
+    const size_t off_moms = take(sizeof(MomMatrix) * nm);
+    const size_t off_smats = take(sizeof(ScaleMatrix) * nm);
+
+    // ---- count problems / maps ---------------------------------------------------
+    size_t nslots = 0;
+    for (const Group& g : groups) nslots = std::max(nslots, g.slots.size());
+    size_t nprob = 0;
+    for (const Group& g : groups)
+        for (const Slot& s : g.slots) nprob += s.size() * g.mats.size();
+    const size_t off_probs = take((f32 ? sizeof(F32Problem) : sizeof(TcProblem)) * std::max<size_t>(nprob, 1));
+    // tiles (upper bound: every tile of every problem)
+    size_t ntiles_max = 0;
+    if (!f32) {
+        for (const Group& g : groups)
+            for (const Slot& s : g.slots)
+                for (const OpDesc& op : s) {
+                    int M, N, K;
+                    OperandGeom A, B;
+                    op_geometry(g, op, M, N, K, A, B);
+                    ntiles_max += static_cast<size_t>((M + tile_m - 1) / tile_m) * ((N + tile_n - 1) / tile_n) *
+                                  g.mats.size();
+                }
+    }
+    const size_t off_tiles = take(sizeof(uint2) * std::max<size_t>(ntiles_max, 1));
+    // tensor maps: at most 2 operands per op per group (deduplicated below)
+    size_t nmaps_max = 0;
+    for (const Group& g : groups)
+        for (const Slot& s : g.slots) nmaps_max += 2 * s.size();
+    const size_t off_maps = take(sizeof(CUtensorMap) * std::max<size_t>(nmaps_max, 1));
+    const size_t need = cursor;
+
+    // ---- arena -----------------------------------------------------------------
+    if (need > arena_bytes) {
+        if (arena_) cudaFree(arena_);
+        arena_ = nullptr;
+        arena_bytes = 0;
+        if (cudaMalloc(&arena_, need) != cudaSuccess) {
+            cudaGetLastError();
+            err = "workspace allocation of " + std::to_string(need) + " bytes failed";
+            return MUON_ERR_NO_MEMORY;
+        }
+        arena_bytes = need;
+    }
+    char* base = static_cast<char*>(arena_);
+    float* d_partials = reinterpret_cast<float*>(base + off_partials);
+    int* d_counters = reinterpret_cast<int*>(base + off_counters);
+    float* d_scale = reinterpret_cast<float*>(base + off_scale);
+    int* d_bad = reinterpret_cast<int*>(base + off_bad);
+    auto buf_ptr = [&](const Group& g, int b, int z) -> char* {
+        return base + g.off[b] + static_cast<size_t>(g.bstride[b]) * z;
+    };
+
+    // ---- momentum / normalise launch -------------------------------------------
+    const int u_dt = f32 ? DT_F32 : DT_BF16;
+    for (int i = 0; i < nm; ++i) {
+        const Group& g = groups[mat_group[i]];
+        MomMatrix& mm = moms[i];
+        mm.g = rq.in[i];
+        mm.m = rq.mom.empty() ? nullptr : rq.mom[i];
+        mm.u = buf_ptr(g, X0, mat_z[i]);
+        mm.rows = rq.rows[i];
+        mm.cols = rq.cols[i];
+        mm.ldu = g.ldx;
+        auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+        mm.vec_ok = (rq.cols[i] % 8 == 0) && mm.ldu == rq.cols[i] && al(mm.g) && al(mm.u) && (!mm.m || al(mm.m));
+    }
+    {
+        LaunchRec lr;
+        lr.kind = LaunchRec::MOM;
+        MomLaunch& L = lr.mom;
+        L.mats = reinterpret_cast<const MomMatrix*>(base + off_moms);
+        L.nmats = nm;
+        L.nchunks = nchunks;
+        L.in_dt = rq.in_dt;
+        L.mom_dt = rq.mom_dt;
+        L.u_dt = u_dt;
+        L.has_momentum = rq.is_step ? 1 : 0;
+        L.nesterov = rq.nesterov;
+        L.mu = rq.mu;
+        L.lr = rq.lr;
+        L.eps = rq.eps;
+        L.partials = d_partials;
+        L.counters = d_counters;
+        L.scale = d_scale;
+        L.bad = d_bad;
+        L.status = status;
+        L.mat_index_base = 0;
+        double elems = 0;
+        for (int i = 0; i < nm; ++i) elems += static_cast<double>(rq.rows[i]) * rq.cols[i];
+        const double per = dtype_size(rq.in_dt) + dtype_size(u_dt) + (rq.is_step ? 2.0 * dtype_size(rq.mom_dt) : 0.0);
+        lr.bytes = elems * per;
+        launches.push_back(lr);
+    }
+
+    // ---- steps == 0: elementwise scale / update ---------------------------------
+    std::vector<ScaleMatrix> smats;
+    if (rq.steps == 0) {
+        long long sc = 0;
+        for (int i = 0; i < nm; ++i) {
+            const Group& g = groups[mat_group[i]];
+            ScaleMatrix s;
+            s.u = buf_ptr(g, X0, mat_z[i]);
+            s.ldu = g.ldx;
+            s.out = rq.out[i];
+            s.rows = rq.rows[i];
+            s.cols = rq.cols[i];
+            s.chunk_begin = sc;
+            s.mat = i;
+            sc += (s.rows * s.cols + kMomChunk - 1) / kMomChunk;
+            smats.push_back(s);
+        }
+        LaunchRec lr;
+        lr.kind = LaunchRec::SCALE;
+        ScaleLaunch& L = lr.sc;
+        L.mats = reinterpret_cast<const ScaleMatrix*>(base + off_smats);
+        L.nmats = nm;
+        L.nchunks = sc;
+        L.u_dt = u_dt;
+        L.out_dt = rq.out_dt;
+        L.update = rq.is_step ? 1 : 0;
+        L.lr = rq.lr;
+        L.scale = d_scale;
+        L.bad = d_bad;
+        launches.push_back(lr);
+    }
+
+    // ---- GEMM launches -------------------------------------------------------------
+    std::vector<TcProblem> tprobs;
+    std::vector<F32Problem> fprobs;
+    std::vector<uint2> tiles;
+    std::vector<CUtensorMap> maps;
+    std::map<std::tuple<int, int, int>, int> map_index;  // (group, buf, box kind)
+    EncodeTiledFn encode = nullptr;
+    if (!f32 && nslots > 0) {
+        encode = get_encoder(err);
+        if (!encode) return MUON_ERR_CUDA;
+    }
+    enum { BOX_KA = 0, BOX_KB = 1, BOX_MN = 2 };
+    auto get_map = [&](int gi, int b, int box) -> int {
+        auto key = std::make_tuple(gi, b, box);
+        auto it = map_index.find(key);
+        if (it != map_index.end()) return it->second;
+        const Group& g = groups[gi];
+        const bool xb = is_x_buf(b);
+        const cuuint64_t inner = xb ? g.cols_w : g.n;
+        const cuuint64_t outer = xb ? g.rows_w : g.n;
+        const cuuint64_t ld = xb ? g.ldx : g.ldn;
+        const int es = dtype_size(g.dt[b]);
+        cuuint64_t dims[3] = {inner, outer, static_cast<cuuint64_t>(g.mats.size())};
+        cuuint64_t strides[2] = {ld * es, static_cast<cuuint64_t>(g.bstride[b])};
+        cuuint32_t boxd[3] = {64, box == BOX_KA ? 128u : (box == BOX_KB ? 256u : 64u), 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUtensorMap m;
+        std::memset(&m, 0, sizeof(m));
+        CUresult r = encode(&m, g.dt[b] == DT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                            3, base + g.off[b], dims, strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            err = "cuTensorMapEncodeTiled failed (" + std::to_string(static_cast<int>(r)) + ")";
+            return -1;
+        }
+        maps.push_back(m);
+        const int idx = static_cast<int>(maps.size()) - 1;
+        map_index[key] = idx;
+        return idx;
+    };
+
+    for (size_t si = 0; si < nslots; ++si) {
+        LaunchRec lr;
+        lr.kind = f32 ? LaunchRec::F32 : LaunchRec::TC;
+        const size_t prob_begin = f32 ? fprobs.size() : tprobs.size();
+        const size_t tile_begin = tiles.size();
+        struct TileRef {
+            uint2 t;
+            int k;
+        };
+        std::vector<TileRef> ltiles;
+        int max_m = 0, max_n = 0;
+        for (size_t gi = 0; gi < groups.size(); ++gi) {
+            const Group& g = groups[gi];
+            if (si >= g.slots.size()) continue;
+            for (const OpDesc& op : g.slots[si]) {
+                int M, N, K;
+                OperandGeom A, B;
+                op_geometry(g, op, M, N, K, A, B);
+                max_m = std::max(max_m, M);
+                max_n = std::max(max_n, N);
+                lr.flops += op_flops(g, op) * g.mats.size();
+                int amap = -1, bmap = -1;
+                if (!f32) {
+                    amap = get_map(static_cast<int>(gi), A.buf, A.mn ? BOX_MN : BOX_KA);
+                    bmap = get_map(static_cast<int>(gi), B.buf, B.mn ? BOX_MN : BOX_KB);
+                    if (amap < 0 || bmap < 0) return MUON_ERR_CUDA;
+                }
+                for (size_t z = 0; z < g.mats.size(); ++z) {
+                    const int mi = g.mats[z];
+                    Epilogue ep;
+                    std::memset(&ep, 0, sizeof(ep));
+                    ep.alpha = op.alpha;
+                    ep.beta = op.beta;
+                    ep.gamma = op.gamma;
+                    ep.delta = op.delta;
+                    ep.sym = op.sym ? 1 : 0;
+                    ep.skip_idx = op.final ? mi : -1;
+                    const float* sc = d_scale + 4 * mi;
+                    if (op.final && rq.is_step)
+                        ep.sigma = sc + (op.sigma == SIG_S ? 2 : 3);  // -lr*s or -lr
+                    else
+                        ep.sigma = op.sigma == SIG_S ? sc : (op.sigma == SIG_S2 ? sc + 1 : nullptr);
+                    auto bind = [&](int b, const void*& p, long long& ld, int& dt) {
+                        if (b < 0) {
+                            p = nullptr;
+                            return;
+                        }
+                        if (b == OUTB) {
+                            p = rq.out[mi];
+                            ld = rq.cols[mi];
+                            dt = rq.out_dt;
+                            return;
+                        }
+                        p = buf_ptr(g, b, static_cast<int>(z));
+                        ld = is_x_buf(b) ? g.ldx : g.ldn;
+                        dt = g.dt[b];
+                    };
+                    const void* tmp = nullptr;
+                    bind(op.c1, ep.c1, ep.ldc1, ep.c1_dt);
+                    bind(op.c2, ep.c2, ep.ldc2, ep.c2_dt);
+                    bind(op.o1, tmp, ep.ldo1, ep.o1_dt);
+                    ep.o1 = const_cast<void*>(tmp);
+                    tmp = nullptr;
+                    bind(op.o2, tmp, ep.ldo2, ep.o2_dt);
+                    ep.o2 = const_cast<void*>(tmp);
+                    if (f32) {
+                        F32Problem p;
+                        std::memset(&p, 0, sizeof(p));
+                        p.M = M;
+                        p.N = N;
+                        p.K = K;
+                        const long long lda = is_x_buf(A.buf) ? g.ldx : g.ldn;
+                        const long long ldb = is_x_buf(B.buf) ? g.ldx : g.ldn;
+                        p.A = reinterpret_cast<const float*>(buf_ptr(g, A.buf, static_cast<int>(z)));
+                        p.a_si = A.mn ? 1 : lda;
+                        p.a_sk = A.mn ? lda : 1;
+                        p.B = reinterpret_cast<const float*>(buf_ptr(g, B.buf, static_cast<int>(z)));
+                        p.b_sk = B.mn ? ldb : 1;
+                        p.b_sj = B.mn ? 1 : ldb;
+                        p.ep = ep;
+                        fprobs.push_back(p);
+                    } else {
+                        TcProblem p;
+                        std::memset(&p, 0, sizeof(p));
+                        p.M = M;
+                        p.N = N;
+                        p.K = K;
+                        p.a_map = amap;
+                        p.b_map = bmap;
+                        p.a_z = static_cast<int>(z);
+                        p.b_z = static_cast<int>(z);
+                        p.a_mn = A.mn ? 1 : 0;
+                        p.b_mn = B.mn ? 1 : 0;
+                        p.fmt = g.dt[A.buf] == DT_F16 ? 0 : 1;
+                        p.ep = ep;
+                        const unsigned pi = static_cast<unsigned>(tprobs.size());
+                        tprobs.push_back(p);
+                        const int tm = (M + tile_m - 1) / tile_m, tn = (N + tile_n - 1) / tile_n;
+                        for (int bi = 0; bi < tm; ++bi)
+                            for (int bj = 0; bj < tn; ++bj) {
+                                if (op.sym && bi * tile_m > bj * tile_n + tile_n - 1) continue;
+                                ltiles.push_back({make_uint2(pi, (static_cast<unsigned>(bi) << 16) | bj), K});
+                            }
+                    }
+                }
+            }
+        }
+        if (f32) {
+            lr.f32.problems = reinterpret_cast<const F32Problem*>(base + off_probs) + prob_begin;
+            lr.f32.nproblems = static_cast<int>(fprobs.size() - prob_begin);
+            lr.f32.max_m = max_m;
+            lr.f32.max_n = max_n;
+            lr.f32.bad = d_bad;
+        } else {
+            // longest K first: a simple LPT order for the persistent CTAs
+            std::stable_sort(ltiles.begin(), ltiles.end(), [](const TileRef& x, const TileRef& y) { return x.k > y.k; });
+            for (const TileRef& t : ltiles) tiles.push_back(t.t);
+            lr.tc.problems = reinterpret_cast<const TcProblem*>(base + off_probs);
+            lr.tc.tiles = reinterpret_cast<const uint2*>(base + off_tiles) + tile_begin;
+            lr.tc.ntiles = static_cast<int>(tiles.size() - tile_begin);
+            lr.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
+            lr.tc.bad = d_bad;
+            lr.tc.status = status;
+            lr.grid = std::min(lr.tc.ntiles, num_sms);
+        }
+        total_flops += lr.flops;
+        launches.push_back(lr);
+    }
+
+    // ---- upload tables -------------------------------------------------------------
+    auto up = [&](size_t off, const void* src, size_t bytes) {
+        if (bytes == 0) return cudaSuccess;
+        return cudaMemcpyAsync(base + off, src, bytes, cudaMemcpyHostToDevice, stream);
+    };
+    cudaError_t e = cudaSuccess;
+    if (e == cudaSuccess) e = up(off_moms, moms.data(), sizeof(MomMatrix) * moms.size());
+    if (e == cudaSuccess) e = up(off_smats, smats.data(), sizeof(ScaleMatrix) * smats.size());
+    if (e == cudaSuccess && !tprobs.empty()) e = up(off_probs, tprobs.data(), sizeof(TcProblem) * tprobs.size());
+    if (e == cudaSuccess && !fprobs.empty()) e = up(off_probs, fprobs.data(), sizeof(F32Problem) * fprobs.size());
+    if (e == cudaSuccess && !tiles.empty()) e = up(off_tiles, tiles.data(), sizeof(uint2) * tiles.size());
+    if (e == cudaSuccess && !maps.empty()) e = up(off_maps, maps.data(), sizeof(CUtensorMap) * maps.size());
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_counters, 0, sizeof(int) * nm, stream);
+    if (e != cudaSuccess) {
+        err = std::string("table upload failed: ") + cudaGetErrorString(e);
+        return MUON_ERR_CUDA;
+    }
+    key_ = make_key(rq);
+    return MUON_OK;
+}
+
+int Plan::run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter, std::string& err) {
+    for (const LaunchRec& lr : launches) {
+        if (prof) prof->before(stream);
+        cudaError_t e = cudaSuccess;
+        switch (lr.kind) {
+            case LaunchRec::MOM: e = launch_momentum_norm(lr.mom, stream); break;
+            case LaunchRec::SCALE: e = launch_scale_apply(lr.sc, stream); break;
+            case LaunchRec::TC: e = launch_gemm_tc(lr.tc, lr.grid, stream); break;
+            case LaunchRec::F32: e = launch_gemm_f32(lr.f32, stream); break;
+        }
+        if (e != cudaSuccess) {
+            err = std::string("kernel launch failed: ") + cudaGetErrorString(e);
+            return MUON_ERR_CUDA;
+        }
+        if (launch_counter) ++*launch_counter;
+        if (prof) prof->after(stream, static_cast<int>(lr.kind), lr.flops, lr.bytes);
+    }
+    return MUON_OK;
+}
+
+}  // namespace muon

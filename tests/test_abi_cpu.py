@@ -1,0 +1,121 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every
+symbol include/muon.h declares, and validates arguments before touching a
+device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import matrix_orthogonalizing_optimizer_step_b200 as mo
+from matrix_orthogonalizing_optimizer_step_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muon.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(_lib.LIB_PATH):
+        from matrix_orthogonalizing_optimizer_step_b200 import build
+        build.build()
+    return mo.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MUON_API\s+[\w\s\*]+?\b(muon_\w+)\s*\(", text)))
+
+
+def test_every_header_symbol_is_exported(lib):
+    names = header_functions()
+    assert len(names) >= 10
+    assert sorted(_lib.EXPORTS) == names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_defaults(lib):
+    assert lib.muon_version() == 10000
+    cfg = mo.muon_default_config()
+    assert cfg["steps"] == 5
+    for t in cfg["coeffs"]:
+        assert t == pytest.approx((3.4445, -4.7750, 2.0315), rel=1e-6)
+    assert cfg["mode"] == mo.MUON_NS_AUTO
+    assert cfg["restart_mask"] == 1 << 2
+    assert cfg["eps"] == pytest.approx(1e-7)
+    assert cfg["momentum_dtype"] == mo.MUON_DTYPE_BF16
+    assert cfg["param_dtype"] == mo.MUON_DTYPE_F32
+
+
+def test_config_roundtrip_and_validation(lib):
+    mo.muon_reset_config()
+    mo.muon_set_config(steps=3, coeffs=[(2, -1.5, 0.5), (3, -4, 2), (1, 0, 0)], mode="gram",
+                       restart_mask=0b10, eps=1e-6)
+    c = mo.muon_get_config()
+    assert c["steps"] == 3 and c["mode"] == mo.MUON_NS_GRAM and c["restart_mask"] == 2
+    assert c["coeffs"][1] == pytest.approx((3, -4, 2))
+    for bad in [dict(steps=17), dict(steps=-1), dict(mode=7), dict(eps=float("nan")),
+                dict(momentum_dtype=5), dict(param_dtype=9)]:
+        with pytest.raises(mo.MuonError) as e:
+            mo.muon_set_config(**bad)
+        assert e.value.code in (mo.MUON_ERR_INVALID_ARG, mo.MUON_ERR_UNSUPPORTED)
+    # a rejected config leaves the installed one untouched
+    assert mo.muon_get_config()["steps"] == 3
+    mo.muon_reset_config()
+    assert lib.muon_set_config(None) == mo.MUON_ERR_INVALID_ARG
+    assert lib.muon_get_config(None) == mo.MUON_ERR_INVALID_ARG
+
+
+def test_orthogonalize_argument_errors(lib):
+    co = (ctypes.c_float * 15)(*([3.4445, -4.775, 2.0315] * 5))
+    dummy = ctypes.c_void_p(0x1000)
+    f = lib.muon_orthogonalize
+    assert f(0, 4, 4, dummy, co, 5, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 0, 4, dummy, co, 5, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, -3, dummy, co, 5, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, None, co, 5, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, dummy, None, 5, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, dummy, co, 17, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, dummy, co, -1, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, dummy, co, 5, 0x4000) == mo.MUON_ERR_INVALID_ARG
+    assert f(1, 4, 4, dummy, co, 5, 9) == mo.MUON_ERR_INVALID_ARG
+    nan = (ctypes.c_float * 3)(float("nan"), 1, 1)
+    assert f(1, 4, 4, dummy, nan, 1, 0) == mo.MUON_ERR_INVALID_ARG
+    assert b"" != lib.muon_last_error()
+
+
+def test_step_argument_errors(lib):
+    vp = ctypes.c_void_p
+    P = (vp * 2)(0x1000, 0x2000)
+    Z = (vp * 2)(0x1000, None)
+    S = (ctypes.c_int * 4)(4, 4, 8, 8)
+    Sbad = (ctypes.c_int * 4)(4, 0, 8, 8)
+    f = lib.muon_step
+    assert f(P, P, P, 0.95, 1, 1e-3, S, 0) == mo.MUON_ERR_INVALID_ARG
+    assert f(None, P, P, 0.95, 1, 1e-3, S, 2) == mo.MUON_ERR_INVALID_ARG
+    assert f(P, P, P, 0.95, 1, 1e-3, None, 2) == mo.MUON_ERR_INVALID_ARG
+    assert f(P, Z, P, 0.95, 1, 1e-3, S, 2) == mo.MUON_ERR_INVALID_ARG
+    assert f(P, P, P, 0.95, 1, 1e-3, Sbad, 2) == mo.MUON_ERR_INVALID_ARG
+    assert f(P, P, P, float("inf"), 1, 1e-3, S, 2) == mo.MUON_ERR_INVALID_ARG
+    assert f(P, P, P, 0.95, 1, float("nan"), S, 2) == mo.MUON_ERR_INVALID_ARG
+
+
+def test_no_device_reports_cuda_error(lib):
+    """Valid arguments on a host without a usable GPU fail with MUON_ERR_CUDA
+    (never a silent CPU fallback)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    co = (ctypes.c_float * 15)(*([3.4445, -4.775, 2.0315] * 5))
+    rc = lib.muon_orthogonalize(1, 8, 8, ctypes.c_void_p(0x1000), co, 5, 0)
+    assert rc == mo.MUON_ERR_CUDA
+    assert b"CUDA" in lib.muon_last_error() or b"device" in lib.muon_last_error()
+
+
+def test_profile_api_without_device(lib):
+    mo.muon_profile_reset()
+    stats = mo.muon_profile_read()
+    assert set(stats) == {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply"}
+    assert all(v["launches"] == 0 for v in stats.values())
+    assert mo.muon_launch_count() >= 0

@@ -1,0 +1,191 @@
+"""GPU parity of the full Muon step (momentum + Newton-Schulz + update)
+against the fp64 oracle, plus determinism, resume and the tracing counters."""
+import numpy as np
+import pytest
+import torch
+
+import matrix_orthogonalizing_optimizer_step_b200 as mo
+from matrix_orthogonalizing_optimizer_step_b200 import workloads as wl
+from oracle import muon_oracle as orc
+from tests._util import TOL_BF16_RELF, TOL_SIGMA, relF, sigma_maxdiff, to64
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+@pytest.fixture(autouse=True)
+def _fresh_config():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    mo.muon_reset_config()
+    yield
+    st, bad = mo.muon_device_status()
+    assert st == mo.MUON_OK, (mo.STATUS_NAMES.get(st), bad)
+    mo.muon_reset_config()
+
+
+def _bf16_round(x64):
+    return torch.from_numpy(x64).float().to(torch.bfloat16).double().numpy()
+
+
+def _expected_momentum(M64, G64, mu, dtype):
+    """fp32 fused multiply-add mu*M + G (exact product in fp64, then one
+    rounding to fp32), then the storage rounding."""
+    m = (np.float64(np.float32(mu)) * M64 + G64).astype(np.float32).astype(np.float64)
+    return _bf16_round(m) if dtype == "bf16" else m
+
+
+def _make_set(shapes, seed, mom_dt="bf16", par_dt="f32"):
+    G = [wl.make_single(r, c, seed + 3 * i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, seed + 3 * i + 1, "student_t3", DEV, mom_dt, 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, seed + 3 * i + 2, "params", DEV, par_dt) for i, (r, c) in enumerate(shapes)]
+    return W, G, M
+
+
+def _run_and_check(shapes, form="auto", mom_dt="bf16", par_dt="f32", nesterov=True, lr=0.1, mu=0.95, seed=1000):
+    mo.muon_set_config(mode=form,
+                       momentum_dtype=mo.MUON_DTYPE_F32 if mom_dt == "f32" else mo.MUON_DTYPE_BF16,
+                       param_dtype=mo.MUON_DTYPE_F32 if par_dt == "f32" else mo.MUON_DTYPE_BF16)
+    W, G, M = _make_set(shapes, seed, mom_dt, par_dt)
+    W64, G64, M64 = [to64(t) for t in W], [to64(t) for t in G], [to64(t) for t in M]
+    mo.muon_step(W, G, M, mu=mu, nesterov=nesterov, lr=lr)
+    torch.cuda.synchronize()
+    for i, (r, c) in enumerate(shapes):
+        n, m = min(r, c), max(r, c)
+        fm = form if form != "auto" else (
+            "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard")
+        W1, M1, O = orc.muon_step(W64[i], G64[i], M64[i], mu, nesterov, lr, form=fm)
+        # momentum buffer: the fp32 update rounded to the storage type
+        got_m = to64(M[i])
+        want_m = _expected_momentum(M64[i], G64[i], mu, mom_dt)
+        exact = np.mean(got_m == want_m)
+        assert exact >= 0.9999, exact
+        # vs the fp64 oracle: one storage rounding of the result plus the fp32
+        # rounding of mu (relative 2^-24 of |mu*M|), which dominates where
+        # mu*M and G cancel
+        tol = (2.0 ** -8 if mom_dt == "bf16" else 2.0 ** -23) * np.abs(M1) + 2.0 ** -22 * np.abs(M64[i])
+        assert np.all(np.abs(got_m - M1) <= tol)
+        # update: recover O from the parameter change
+        got_w = to64(W[i])
+        if par_dt == "f32":
+            O_gpu = (W64[i] - got_w) / lr
+            assert relF(O_gpu, O) <= TOL_BF16_RELF, (shapes[i], relF(O_gpu, O))
+            assert sigma_maxdiff(O_gpu, O) <= TOL_SIGMA
+        else:
+            want = _bf16_round(W1)
+            # bf16 parameters: within one bf16 ulp of the rounded oracle update
+            assert np.max(np.abs(got_w - want) / np.maximum(np.abs(want), 1e-3)) <= 2 ** -7
+
+
+SHAPES = [(256, 768), (768, 256), (200, 200), (136, 520), (520, 136), (64, 64)]
+
+
+@pytest.mark.parametrize("form", ["standard", "gram", "auto"])
+def test_step_forms(form):
+    _run_and_check(SHAPES, form=form)
+
+
+def test_step_no_nesterov():
+    _run_and_check(SHAPES[:3], nesterov=False)
+
+
+def test_step_fp32_momentum():
+    _run_and_check(SHAPES[:4], mom_dt="f32")
+
+
+def test_step_bf16_params():
+    _run_and_check(SHAPES[:4], par_dt="bf16", lr=0.5)
+
+
+def test_step_unaligned_columns():
+    _run_and_check([(37, 91), (91, 37), (13, 200)], form="auto")
+
+
+def test_step_zero_lr_leaves_params():
+    W, G, M = _make_set([(96, 160)], 77)
+    W0 = W[0].clone()
+    mo.muon_step(W, G, M, mu=0.9, nesterov=True, lr=0.0)
+    torch.cuda.synchronize()
+    assert torch.equal(W[0], W0)
+
+
+def test_step_nonfinite_gradient_leaves_param():
+    W, G, M = _make_set([(64, 192), (96, 96)], 88)
+    G[1][5, 7] = float("nan")
+    W1 = W[1].clone()
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.1)
+    st, bad = mo.muon_device_status()
+    assert st == mo.MUON_ERR_NONFINITE and bad == 1
+    assert torch.equal(W[1], W1)
+    mo.muon_reset_config()
+
+
+def test_step_deterministic_and_resumable():
+    """Two identical runs are bitwise equal; resuming from saved (W, M) after
+    k steps equals the uninterrupted run (the library keeps no hidden state)."""
+    shapes = [(256, 768), (768, 256), (128, 128)]
+
+    def run(nsteps, W, G, M):
+        for _ in range(nsteps):
+            mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.02)
+        torch.cuda.synchronize()
+
+    Wa, G, Ma = _make_set(shapes, 300)
+    Wb, Mb = [t.clone() for t in Wa], [t.clone() for t in Ma]
+    run(3, Wa, G, Ma)
+    run(3, Wb, G, Mb)
+    for x, y in zip(Wa + Ma, Wb + Mb):
+        assert torch.equal(x, y)
+    Wc, _, Mc = _make_set(shapes, 300)
+    run(2, Wc, G, Mc)
+    saved_W = [t.cpu().clone() for t in Wc]
+    saved_M = [t.cpu().clone() for t in Mc]
+    Wd = [t.to(DEV) for t in saved_W]
+    Md = [t.to(DEV) for t in saved_M]
+    run(1, Wd, G, Md)
+    for x, y in zip(Wa + Ma, Wd + Md):
+        assert torch.equal(x, y)
+
+
+def test_profile_counts_match_oracle_flops():
+    shapes = [(256, 768), (768, 256), (512, 512)]
+    W, G, M = _make_set(shapes, 500)
+    mo.muon_set_config(mode="auto")
+    mo.muon_step(W, G, M)  # builds the plan
+    torch.cuda.synchronize()
+    mo.muon_profile_reset()
+    mo.muon_profile_enable(True)
+    n0 = mo.muon_launch_count()
+    mo.muon_step(W, G, M)
+    prof = mo.muon_profile_read()
+    mo.muon_profile_enable(False)
+    launches = mo.muon_launch_count() - n0
+    want = 0
+    for r, c in shapes:
+        n, m = min(r, c), max(r, c)
+        want += min(orc.ns_flops(n, m, 5, "gram"), orc.ns_flops(n, m, 5, "standard"))
+    assert prof["gemm_tc"]["flops"] == pytest.approx(want, rel=1e-9)
+    assert prof["momentum_norm"]["launches"] == 1
+    assert launches == prof["gemm_tc"]["launches"] + 1
+    assert prof["gemm_tc"]["total_ms"] > 0
+
+
+def test_gpt2_set_full_parity():
+    """Workload 2 (GPT-2 124M Muon set, 48 matrices) at full size: every
+    matrix against the oracle."""
+    w = wl.WORKLOADS[2]
+    W = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=DEV) for i in range(w.count)]
+    G = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=DEV) for i in range(w.count)]
+    M = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=DEV) for i in range(w.count)]
+    W64, G64, M64 = [to64(t) for t in W], [to64(t) for t in G], [to64(t) for t in M]
+    lr = 6e-4
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=lr)
+    torch.cuda.synchronize()
+    worst = 0.0
+    for i, (r, c) in enumerate(w.shapes):
+        _, _, O = orc.muon_step(W64[i], G64[i], M64[i], 0.95, True, lr, form="standard")
+        O_gpu = (W64[i] - to64(W[i])) / lr
+        e = relF(O_gpu, O)
+        worst = max(worst, e)
+        # the update is recovered from an fp32 difference: allow its rounding
+        assert e <= TOL_BF16_RELF + 2e-3, (i, w.shapes[i], e)
+    print("gpt2 worst relF", worst)

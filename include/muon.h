@@ -146,6 +146,39 @@ MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* c
 MUON_API int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
               float lr, const int* shape_list, int count);
 
+/* ---- allocation-free normalisation ---------------------------------------
+ *
+ * The pages have no counterpart to this call: it exists for callers that
+ * cannot allocate device memory -- code whose device memory belongs to a
+ * framework's allocator or to a fixed budget reserved up front, and
+ * latency-critical paths where a cudaMalloc (which may synchronise the
+ * device) is not acceptable.
+ *
+ * muon_normalize_noalloc -- Y_i = X_i / (||X_i||_F + eps) for batch matrices
+ * of m x n, the same result as muon_orthogonalize with steps = 0.  It calls no
+ * cudaMalloc, cudaFree or allocating library routine: its scratch (per-chunk
+ * partial sums, per-matrix ticket counters and scales) is a file-scope device
+ * array of fixed size, MUON_NOALLOC_MAX_CHUNKS * 4 + MUON_NOALLOC_MAX_MATRICES
+ * * 8 bytes (about 264 KiB), which every GPU that loads the library holds
+ * until the process exits.
+ * batch, m, n  >= 1; batch <= MUON_NOALLOC_MAX_MATRICES and
+ *              batch * ceil(m*n / 8192) <= MUON_NOALLOC_MAX_CHUNKS, else
+ *              MUON_ERR_INVALID_ARG (nothing is enqueued)
+ * X, Y         device pointers to batch contiguous row-major m x n matrices
+ *              of `dtype` (MUON_DTYPE_BF16 or MUON_DTYPE_F32); Y may equal X
+ * eps          finite, >= 0
+ * Work is enqueued on the bound stream.  The first call on a device looks up
+ * the array's device address on that device (once, with that device
+ * current); make that first call before any stream capture.  Every call
+ * shares the array and it keeps the last call's contents: each call clears
+ * the counters it uses, and calls that overlap on the GPU (other streams,
+ * other threads) race on it.  A matrix whose norm is not finite leaves its Y
+ * untouched.
+ */
+#define MUON_NOALLOC_MAX_MATRICES 1024
+#define MUON_NOALLOC_MAX_CHUNKS 65536 /* chunks of 8192 elements: 512 Mi elements in one call */
+MUON_API int muon_normalize_noalloc(int batch, int m, int n, const void* X, void* Y, int dtype, float eps);
+
 /* ---- tracing ------------------------------------------------------------ */
 
 typedef struct muon_kernel_stats {

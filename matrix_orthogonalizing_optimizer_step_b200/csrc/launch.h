@@ -62,4 +62,8 @@ struct ScaleLaunch {
 };
 cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream);
 
+// The stream bound by muon_set_stream, and the message muon_last_error returns.
+cudaStream_t bound_stream();
+void set_last_error(const char* msg);
+
 }  // namespace muon

@@ -199,6 +199,11 @@ int check_device(DeviceState** ds, bool need_tc) {
 
 }  // namespace
 
+namespace muon {
+cudaStream_t bound_stream() { return g_stream; }
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace muon
+
 extern "C" {
 
 int muon_version(void) { return MUON_VERSION; }

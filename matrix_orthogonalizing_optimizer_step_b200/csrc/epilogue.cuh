@@ -108,11 +108,28 @@ __device__ __forceinline__ void store_row32(void* base, int dt, long long ld, lo
         if (j >= jmin && j < nvalid) st_elem(base, dt, off + j, v[j]);
 }
 
+// C1 row segment fetched ahead of its use (16-bit C1, aligned, fully in range).
+struct Raw32 {
+    uint4 q[4];
+    int ok;
+};
+
+__device__ __forceinline__ void prefetch_row32(const Epilogue& ep, int M, int N, long long row, int col0, Raw32& r) {
+    r.ok = 0;
+    if (!ep.c1 || ep.c1_dt == DT_F32 || row >= M || col0 + 32 > N) return;
+    const uint16_t* p = static_cast<const uint16_t*>(ep.c1) + row * ep.ldc1 + col0;
+    if (reinterpret_cast<uintptr_t>(p) & 15) return;
+    const uint4* v = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) r.q[i] = v[i];
+    r.ok = 1;
+}
+
 // Apply the fused epilogue to a 32-column row segment of the accumulator:
 // row `row`, columns col0 .. col0 + 31 of an M x N output.  `sig` is the
 // problem's sigma (already loaded).
 __device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, int M, int N, long long row, int col0,
-                                               float* acc) {
+                                               float* acc, const Raw32* pre = nullptr) {
     if (row >= M) return;
     const int nvalid = min(32, N - col0);
     if (nvalid <= 0) return;
@@ -121,7 +138,12 @@ __device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, in
     if (jmin >= nvalid) return;
     float t1[32];
     if (ep.c1) {
-        load_row32(ep.c1, ep.c1_dt, ep.ldc1, row, col0, nvalid, t1);
+        if (pre && pre->ok) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) unpack8(pre->q[i], ep.c1_dt, t1 + 8 * i);
+        } else {
+            load_row32(ep.c1, ep.c1_dt, ep.ldc1, row, col0, nvalid, t1);
+        }
 #pragma unroll
         for (int j = 0; j < 32; ++j) acc[j] = fmaf(ep.beta, t1[j], ep.alpha * acc[j]);
     } else {

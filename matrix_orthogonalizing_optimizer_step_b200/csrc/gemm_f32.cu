@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(256) gemm_f32_kernel(const F32Launch L) {
         }
         __syncthreads();
     }
-    const Epilogue& ep = P.ep;
+    const Epilogue ep = P.ep;  // local copy: no reloads after global stores
     if (ep.skip_idx >= 0 && L.bad[ep.skip_idx]) return;
     const float sig = ep.sigma ? *ep.sigma : 1.f;
 #pragma unroll

@@ -1,20 +1,31 @@
-// Persistent grouped tensor-core GEMM for sm_100a with a fused epilogue.
+// Persistent grouped tensor-core GEMM for sm_100a with a fused epilogue,
+// run by CTA pairs (cluster of 2, tcgen05 cta_group::2).
 //
-// Every product of the Newton-Schulz chain (X X^T, polynomial-in-R products,
-// the final Q X / B X) is one TcProblem; a launch runs a list of 128 x 256
-// output tiles drawn from many problems (matrices of different shapes).
+// Every product of the Newton-Schulz chain (X X^T, the polynomial-in-R
+// products, the final Q X / B X) is one TcProblem; a launch walks a list of
+// 256 x 256 output tiles drawn from many problems (matrices of different
+// shapes).  A CTA pair owns one tile at a time: CTA r holds rows
+// [128 r, 128 r + 128) of A and of B (B split along N), the leader CTA (r = 0)
+// issues M=256 N=256 K=16 MMAs that read both CTAs' shared memory, and each
+// CTA's TMEM receives its 128 rows of the fp32 accumulator.  Per CTA and
+// 64-wide K slice this moves 32 KB of operands for 4.2 MFLOP, a third less
+// than a single-CTA 128 x 256 tile.
 //
-//   warp 0      TMA producer: 64-wide K slices of A (128 rows) and B (256 rows)
-//               into a 4-stage shared-memory ring (128-byte swizzle, no multicast)
-//   warp 1      TMEM owner and MMA issuer: tcgen05.mma kind::f16, M=128 N=256
-//               K=16, fp32 accumulators in TMEM, two accumulator slots
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, fused combine
+//   warp 0      TMA producer (both CTAs): 64-wide K slices of its halves of A
+//               and B into a 6-stage ring (128-byte swizzle, no multicast);
+//               the transaction bytes of both CTAs land on the leader's barrier
+//   warp 1      TMEM owner (both CTAs) and MMA issuer (leader only):
+//               two 256-column fp32 accumulators (double-buffered)
+//   warps 2..9  epilogue: tcgen05.ld of 32-column slices, fused combine
 //               sigma*(alpha*acc + beta*C1) + gamma*C2 + delta*I, stores
-//               (mirrored for symmetric outputs)
 //
-// The epilogue of tile i overlaps the main loop of tile i+1 (double-buffered
-// TMEM).  Every wait is bounded: on expiry the kernel records a timeout in the
-// device status word, drains its own copies and MMAs, frees TMEM and exits.
+// Symmetric outputs (X X^T and every product of polynomials in R) are only
+// computed and stored for the upper 256 x 256 tiles; consumers read a lower
+// block through the transposed tensor map of the mirrored upper tile, so no
+// transposed (mirror) store is ever issued.
+//
+// Every wait is bounded: on expiry the kernel records a timeout in the device
+// status word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -25,52 +36,73 @@
 namespace muon {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128;        // rows of A (and of the output) per CTA
+constexpr int BMP = 2 * BM;    // rows per CTA pair
+constexpr int BN = 256;        // output columns per tile
+constexpr int BNH = BN / 2;    // B rows (N) loaded per CTA
+constexpr int BK = 64;
+constexpr int STAGES = 6;
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int B_BYTES = BNH * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;  // 2 accumulators x 256 fp32 columns
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
 
 struct Shared {
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t tfull[2];
-    uint64_t tempty[2];
+    uint64_t full[STAGES];   // leader: both CTAs' operand bytes landed
+    uint64_t empty[STAGES];  // each CTA: its slot may be refilled (leader's MMA commit)
+    uint64_t tfull[2];       // each CTA: accumulator ready (leader's MMA commit)
+    uint64_t tempty[2];      // leader: all 2 x EPI_WARPS epilogue warps drained the accumulator
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
+
+// Symmetric operands are stored as upper 256 x 256 tiles: the 64-wide K slice
+// kb of the 256-row block `blk` lies in a lower (unstored) tile when blk > kb/4.
+__device__ __forceinline__ bool slice_is_lower(int blk, int kb) { return blk > (kb * BK) / BN; }
 
 __device__ __forceinline__ void record_timeout(Shared* sh, DeviceStatus* st) {
     atomicOr(&st->bits, ST_TIMEOUT);
     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
 }
 
-__device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh) {
+__device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t rank, int pair, int npairs) {
     volatile int* abort_flag = &sh->abort;
+    const bool leader = rank == 0;
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t issued = 0;  // number of stage fills issued
+    uint32_t issued = 0;
     bool ok = true;
     int last_a = -1, last_b = -1;
-    for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+    for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const uint2 tile = L.tiles[t];
-        const TcProblem& P = L.problems[tile.x];
+        // register copies: the asm statements below clobber memory, so fields
+        // read through the problem table would be reloaded inside the K loop
+        const TcProblem& Pg = L.problems[tile.x];
+        const int a_z = Pg.a_z, b_z = Pg.b_z, K = Pg.K;
+        const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, a_sym = Pg.a_sym, b_sym = Pg.b_sym;
         const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
-        const CUtensorMap* ma = L.maps + P.a_map;
-        const CUtensorMap* mb = L.maps + P.b_map;
-        if (P.a_map != last_a) {
+        const CUtensorMap* ma = L.maps + Pg.a_map;
+        const CUtensorMap* mb = L.maps + Pg.b_map;
+        const CUtensorMap* ma_t = a_sym ? L.maps + Pg.a_map_t : ma;
+        const CUtensorMap* mb_t = b_sym ? L.maps + Pg.b_map_t : mb;
+        if (Pg.a_map != last_a) {
             tma_map_acquire(ma);
-            last_a = P.a_map;
+            if (a_sym) tma_map_acquire(ma_t);
+            last_a = Pg.a_map;
         }
-        if (P.b_map != last_b) {
+        if (Pg.b_map != last_b) {
             tma_map_acquire(mb);
-            last_b = P.b_map;
+            if (b_sym) tma_map_acquire(mb_t);
+            last_b = Pg.b_map;
         }
-        const int nk = (P.K + BK - 1) / BK;
+        const int arow = bi * BMP + static_cast<int>(rank) * BM;   // this CTA's A rows
+        const int brow = bj * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows (N)
+        const int nk = (K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) {
                 ok = false;
@@ -78,20 +110,25 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh) {
             }
             uint8_t* sa = tiles_smem + stage * STAGE_BYTES;
             uint8_t* sb = sa + A_BYTES;
-            mbar_arrive_expect_tx(&sh->full[stage], STAGE_BYTES);
-            if (!P.a_mn) {
-                tma_load_3d(sa, ma, &sh->full[stage], kb * BK, bi * BM, P.a_z);
+            const uint32_t full_leader = map_to_cta(smem_u32(&sh->full[stage]), 0);
+            if (leader) mbar_arrive_expect_tx(&sh->full[stage], 2 * STAGE_BYTES);
+            // a K slice of a symmetric operand below its stored upper tiles is
+            // read transposed from the mirrored tile (same values)
+            const bool a_t = a_mn || (a_sym && slice_is_lower(bi, kb));
+            const bool b_t = b_mn || (b_sym && slice_is_lower(bj, kb));
+            if (!a_t) {
+                tma_load_3d_pair(sa, ma, full_leader, kb * BK, arow, a_z);
             } else {
 #pragma unroll
                 for (int j = 0; j < BM / 64; ++j)
-                    tma_load_3d(sa + j * MN_BLOCK_BYTES, ma, &sh->full[stage], bi * BM + 64 * j, kb * BK, P.a_z);
+                    tma_load_3d_pair(sa + j * MN_BLOCK_BYTES, ma_t, full_leader, arow + 64 * j, kb * BK, a_z);
             }
-            if (!P.b_mn) {
-                tma_load_3d(sb, mb, &sh->full[stage], kb * BK, bj * BN, P.b_z);
+            if (!b_t) {
+                tma_load_3d_pair(sb, mb, full_leader, kb * BK, brow, b_z);
             } else {
 #pragma unroll
-                for (int j = 0; j < BN / 64; ++j)
-                    tma_load_3d(sb + j * MN_BLOCK_BYTES, mb, &sh->full[stage], bj * BN + 64 * j, kb * BK, P.b_z);
+                for (int j = 0; j < BNH / 64; ++j)
+                    tma_load_3d_pair(sb + j * MN_BLOCK_BYTES, mb_t, full_leader, brow + 64 * j, kb * BK, b_z);
             }
             ++issued;
             if (++stage == STAGES) {
@@ -101,19 +138,22 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh) {
         }
     }
     if (!ok) record_timeout(sh, L.status);
-    // Drain: every issued fill must have landed before the CTA exits.  Fill i
-    // used stage i % STAGES with phase parity (i / STAGES) & 1.
-    const uint32_t first = issued > STAGES ? issued - STAGES : 0;
-    int never = 0;
-    for (uint32_t i = first; i < issued; ++i) {
-        if (!mbar_wait(&sh->full[i % STAGES], (i / STAGES) & 1u, &never)) {
-            atomicOr(&L.status->bits, ST_TIMEOUT);
-            break;
+    // Drain (leader): the last fills of every stage must have landed before
+    // the pair exits.  Fill i used stage i % STAGES, phase parity (i / STAGES) & 1.
+    if (leader) {
+        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+        int never = 0;
+        for (uint32_t i = first; i < issued; ++i) {
+            if (!mbar_wait(&sh->full[i % STAGES], (i / STAGES) & 1u, &never)) {
+                atomicOr(&L.status->bits, ST_TIMEOUT);
+                break;
+            }
         }
     }
 }
 
-__device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base) {
+__device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base, int pair,
+                           int npairs) {
     volatile int* abort_flag = &sh->abort;
     int stage = 0;
     uint32_t phase = 0;
@@ -122,16 +162,18 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     bool ok = true;
     bool issued_any = false;
     const uint32_t tiles_base = smem_u32(tiles_smem);
-    for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+    for (int t = pair; t < L.ntiles && ok; t += npairs) {
         const uint2 tile = L.tiles[t];
-        const TcProblem& P = L.problems[tile.x];
-        const int nk = (P.K + BK - 1) / BK;
+        const TcProblem& Pg = L.problems[tile.x];
+        const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, K = Pg.K, fmt = Pg.fmt;  // registers (see producer)
+        const int a_sym = Pg.a_sym, b_sym = Pg.b_sym;
+        const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
+        const int nk = (K + BK - 1) / BK;
         if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag)) {
             ok = false;
             break;
         }
         tc_fence_after();
-        const uint32_t idesc = make_instr_desc(P.fmt, P.a_mn, P.b_mn, BM, BN);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait(&sh->full[stage], phase, abort_flag)) {
@@ -141,25 +183,28 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             tc_fence_after();
             const uint32_t a_addr = tiles_base + stage * STAGE_BYTES;
             const uint32_t b_addr = a_addr + A_BYTES;
+            const int a_t = (a_mn || (a_sym && slice_is_lower(bi, kb))) ? 1 : 0;  // as loaded by the producer
+            const int b_t = (b_mn || (b_sym && slice_is_lower(bj, kb))) ? 1 : 0;
+            const uint32_t idesc = make_instr_desc(fmt, a_t, b_t, BMP, BN);
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
                 // K-major: advance 16 elements (32 B) inside the swizzled row;
                 // MN-major: advance 16 k-rows (two 8-row groups of 1024 B).
-                const uint64_t ad = P.a_mn ? make_smem_desc(a_addr + k * 2048, MN_BLOCK_BYTES, 1024)
-                                           : make_smem_desc(a_addr + k * 32, 16, 1024);
-                const uint64_t bd = P.b_mn ? make_smem_desc(b_addr + k * 2048, MN_BLOCK_BYTES, 1024)
-                                           : make_smem_desc(b_addr + k * 32, 16, 1024);
-                umma_f16(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                const uint64_t ad = a_t ? make_smem_desc(a_addr + k * 2048, MN_BLOCK_BYTES, 1024)
+                                        : make_smem_desc(a_addr + k * 32, 16, 1024);
+                const uint64_t bd = b_t ? make_smem_desc(b_addr + k * 2048, MN_BLOCK_BYTES, 1024)
+                                        : make_smem_desc(b_addr + k * 32, 16, 1024);
+                umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
             }
             issued_any = true;
-            umma_commit(&sh->empty[stage]);  // frees the smem slot once these MMAs finish
+            umma_commit_pair(&sh->empty[stage], 0x3);  // both CTAs may refill this slot
             if (++stage == STAGES) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
         if (!ok) break;
-        umma_commit(&sh->tfull[acc]);  // accumulator ready for the epilogue
+        umma_commit_pair(&sh->tfull[acc], 0x3);  // accumulator ready in both CTAs
         if (++acc == 2) {
             acc = 0;
             acc_phase ^= 1u;
@@ -170,49 +215,63 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
         if (issued_any) {
             // wait for this thread's MMAs before TMEM is released
             int never = 0;
-            umma_commit(&sh->drain);
+            umma_commit_pair(&sh->drain, 0x1);
             if (!mbar_wait(&sh->drain, 0, &never)) atomicOr(&L.status->bits, ST_TIMEOUT);
         }
     }
 }
 
-__device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base, int warp, int lane) {
+__device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base, int warp, int lane, uint32_t rank,
+                               int pair, int npairs) {
     volatile int* abort_flag = &sh->abort;
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;  // column half of the tile
+    const uint32_t tempty_leader[2] = {map_to_cta(smem_u32(&sh->tempty[0]), 0),
+                                       map_to_cta(smem_u32(&sh->tempty[1]), 0)};
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
+    for (int t = pair; t < L.ntiles; t += npairs) {
         const uint2 tile = L.tiles[t];
-        const TcProblem& P = L.problems[tile.x];
+        // Local copies: the epilogue stores to global memory, so fields read
+        // through a reference into the problem table would be reloaded after
+        // every store (the compiler cannot rule out aliasing).
+        const Epilogue ep = L.problems[tile.x].ep;
+        const int PM = L.problems[tile.x].M, PN = L.problems[tile.x].N;
         const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
+        const bool skip = ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0;
+        const float sig = ep.sigma ? *ep.sigma : 1.f;
+        const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;
+        const long long row = row0 + lane;
+        const int cbase = bj * BN + half * (BN / 2);
+        // prefetch the C1 row segment of the first slice while the MMAs run
+        Raw32 pre[2];
+        prefetch_row32(ep, PM, PN, row, cbase, pre[0]);
         if (!mbar_wait(&sh->tfull[acc], acc_phase, abort_flag)) {
             if (lane == 0) record_timeout(sh, L.status);
             break;
         }
         tc_fence_after();
-        const Epilogue& ep = P.ep;
-        const bool skip = ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0;
-        const float sig = ep.sigma ? *ep.sigma : 1.f;
-        const long long row0 = static_cast<long long>(bi) * BM + q * 32;
-        const long long row = row0 + lane;
-        for (int c = 0; c < BN; c += 32) {
-            const int col0 = bj * BN + c;
-            if (col0 >= P.N) break;                          // warp-uniform
-            if (ep.sym && row0 > col0 + 31) continue;        // warp-uniform: strictly below the diagonal
+#pragma unroll
+        for (int c = 0; c < BN / 2; c += 32) {
+            const int col0 = cbase + c;
+            const int cur = (c / 32) & 1;
+            if (c + 32 < BN / 2) prefetch_row32(ep, PM, PN, row, col0 + 32, pre[cur ^ 1]);
+            if (col0 >= PN) continue;  // warp-uniform
             uint32_t r[32];
             __syncwarp();
-            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c, r);
+            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * (BN / 2) + c,
+                               r);
             tmem_wait_ld();
             if (!skip) {
                 float v[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                epilogue_row32(ep, sig, P.M, P.N, row, col0, v);
+                epilogue_row32(ep, sig, PM, PN, row, col0, v, &pre[cur]);
             }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sh->tempty[acc]);
+        if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
         if (++acc == 2) {
             acc = 0;
             acc_phase ^= 1u;
@@ -220,12 +279,15 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
     }
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcLaunch L) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ TcLaunch L) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem =
         reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     Shared* sh = reinterpret_cast<Shared*>(tiles_smem + STAGES * STAGE_BYTES);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const uint32_t rank = cluster_cta_rank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -234,42 +296,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_tc_kernel(const __grid_co
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sh->tfull[a], 1);
-            mbar_init(&sh->tempty[a], 4);  // one arrival per epilogue warp
+            mbar_init(&sh->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
         }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&sh->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&sh->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
+    cluster_sync_all();  // the peer's barriers exist before anyone signals them
     tc_fence_after();
     const uint32_t tmem_base = sh->tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) producer(L, tiles_smem, sh);
+        if (lane == 0) producer(L, tiles_smem, sh, rank, pair, npairs);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(L, tiles_smem, sh, tmem_base);
+        if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base, pair, npairs);
     } else {
-        epilogue_warps(L, sh, tmem_base, warp, lane);
+        epilogue_warps(L, sh, tmem_base, warp, lane, rank, pair, npairs);
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync_all();  // no CTA leaves while its peer may still touch its memory or TMEM
     tc_fence_after();
     if (warp == 1) {
         __syncwarp();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
 }  // namespace
 
 size_t gemm_tc_smem_bytes() { return SMEM_BYTES; }
-int gemm_tc_tile_m() { return BM; }
+int gemm_tc_tile_m() { return BMP; }
 int gemm_tc_tile_n() { return BN; }
 
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream) {

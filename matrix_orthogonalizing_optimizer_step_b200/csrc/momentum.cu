@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     __shared__ int is_last;
     const long long chunk = blockIdx.x;
     const int mi = find_matrix(L.nmats, chunk, L.mats);
-    const MomMatrix& Mx = L.mats[mi];
+    const MomMatrix Mx = L.mats[mi];  // local copy: no reloads after global stores
     const long long numel = Mx.rows * Mx.cols;
     const long long e0 = (chunk - Mx.chunk_begin) * kMomChunk;
     const float mu = L.mu;
@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(kThreads) scale_apply_kernel(const ScaleLaunch
         else
             hi = mid - 1;
     }
-    const ScaleMatrix& S = L.mats[lo];
+    const ScaleMatrix S = L.mats[lo];
     if (L.bad[S.mat]) return;
     const float s = L.scale[4 * S.mat];
     const long long numel = S.rows * S.cols;

@@ -5,6 +5,8 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <deque>
 #include <memory>
@@ -151,10 +153,18 @@ struct Profiler : ProfileSink {
         cur = nullptr;
     }
     void fold() {
+        // MUON_PROFILE_VERBOSE=1 prints every traced launch (position in the
+        // call, kind, ms, algorithmic TFLOP/s or GB/s) to stderr.
+        static const bool verbose = std::getenv("MUON_PROFILE_VERBOSE") != nullptr;
+        int pos = 0;
         for (Pending& p : pending) {
             float ms = 0.f;
             cudaEventSynchronize(p.b);
             cudaEventElapsedTime(&ms, p.a, p.b);
+            if (verbose)
+                std::fprintf(stderr, "muon launch %3d kind %d %9.4f ms %8.2f TFLOP/s %8.1f GB/s\n", pos, p.kind, ms,
+                             ms > 0 ? p.flops / (ms * 1e-3) / 1e12 : 0.0, ms > 0 ? p.bytes / (ms * 1e-3) / 1e9 : 0.0);
+            ++pos;
             muon_kernel_stats& st = stats[p.kind];
             st.launches += 1;
             st.total_ms += ms;

@@ -21,8 +21,9 @@ struct DeviceStatus {
 //   v = sigma * (alpha * acc + beta * C1) + gamma * C2 + delta * [row == col]
 // sigma is 1 when sigma_ptr is null.  sigma == 0 forces the first term to 0
 // (so a non-finite accumulator of a rejected matrix does not leak through).
-// With sym, only elements with row <= col are produced and each is also
-// written at the mirrored position (col, row).
+// With sym (fp32 check path only), only elements with row <= col are
+// produced and each is also written at the mirrored position (col, row); the
+// tensor-core path instead stores symmetric outputs as upper tiles.
 struct Epilogue {
     float alpha, beta, gamma, delta;
     const float* sigma;  // per-matrix scale (device) or null
@@ -37,12 +38,19 @@ struct Epilogue {
 // One tensor-core GEMM problem D[M x N] = A[M x K] * B[K x N] (B given as N x K
 // "rows" in tcgen05 terms).  Operands are read by TMA through tensor maps in
 // global memory; a_mn / b_mn select the MN-major (transposed) smem layout.
+//
+// Symmetric n x n matrices are stored as their upper 256 x 256 tiles only
+// (diagonal tiles in full).  An operand marked a_sym / b_sym is such a matrix:
+// a 64-wide K slice that falls in a lower tile is fetched from the mirrored
+// upper tile through the transposed (MN-major) map a_map_t / b_map_t.
 struct TcProblem {
     int M, N, K;
-    int a_map, b_map;  // indices into the launch's tensor-map array
-    int a_z, b_z;      // batch coordinate (3rd tensor-map dimension)
-    int a_mn, b_mn;    // 1: operand is MN-major in memory
-    int fmt;           // 0 = f16 operands, 1 = bf16 operands
+    int a_map, b_map;      // indices into the launch's tensor-map array
+    int a_map_t, b_map_t;  // MN-major maps of symmetric operands (else -1)
+    int a_z, b_z;          // batch coordinate (3rd tensor-map dimension)
+    int a_mn, b_mn;        // 1: operand is MN-major in memory
+    int a_sym, b_sym;      // 1: operand is an upper-stored symmetric matrix
+    int fmt;               // 0 = f16 operands, 1 = bf16 operands
     int pad_;
     Epilogue ep;
 };

@@ -476,10 +476,11 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                 }
     }
     const size_t off_tiles = take(sizeof(uint2) * std::max<size_t>(ntiles_max, 1));
-    // tensor maps: at most 2 operands per op per group (deduplicated below)
+    // tensor maps: at most 2 operands per op per group, each with a transposed
+    // map when symmetric (deduplicated below)
     size_t nmaps_max = 0;
     for (const Group& g : groups)
-        for (const Slot& s : g.slots) nmaps_max += 2 * s.size();
+        for (const Slot& s : g.slots) nmaps_max += 4 * s.size();
     const size_t off_maps = take(sizeof(CUtensorMap) * std::max<size_t>(nmaps_max, 1));
     const size_t need = cursor;
 
@@ -602,7 +603,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         const int es = dtype_size(g.dt[b]);
         cuuint64_t dims[3] = {inner, outer, static_cast<cuuint64_t>(g.mats.size())};
         cuuint64_t strides[2] = {ld * es, static_cast<cuuint64_t>(g.bstride[b])};
-        cuuint32_t boxd[3] = {64, box == BOX_KA ? 128u : (box == BOX_KB ? 256u : 64u), 1};
+        // K-major operands: 64 (K) x 128 rows per CTA; MN-major: 64 (MN) x 64 (K)
+        cuuint32_t boxd[3] = {64, box == BOX_MN ? 64u : 128u, 1};
         cuuint32_t estr[3] = {1, 1, 1};
         CUtensorMap m;
         std::memset(&m, 0, sizeof(m));
@@ -641,11 +643,16 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                 max_m = std::max(max_m, M);
                 max_n = std::max(max_n, N);
                 lr.flops += op_flops(g, op) * g.mats.size();
-                int amap = -1, bmap = -1;
+                int amap = -1, bmap = -1, amap_t = -1, bmap_t = -1;
+                // n x n operands are symmetric, stored as upper tiles by the
+                // tensor-core path: their lower blocks are read transposed
+                const bool a_sym = !f32 && !is_x_buf(A.buf), b_sym = !f32 && !is_x_buf(B.buf);
                 if (!f32) {
                     amap = get_map(static_cast<int>(gi), A.buf, A.mn ? BOX_MN : BOX_KA);
                     bmap = get_map(static_cast<int>(gi), B.buf, B.mn ? BOX_MN : BOX_KB);
-                    if (amap < 0 || bmap < 0) return MUON_ERR_CUDA;
+                    if (a_sym) amap_t = get_map(static_cast<int>(gi), A.buf, BOX_MN);
+                    if (b_sym) bmap_t = get_map(static_cast<int>(gi), B.buf, BOX_MN);
+                    if (amap < 0 || bmap < 0 || (a_sym && amap_t < 0) || (b_sym && bmap_t < 0)) return MUON_ERR_CUDA;
                 }
                 for (size_t z = 0; z < g.mats.size(); ++z) {
                     const int mi = g.mats[z];
@@ -709,12 +716,17 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                         p.K = K;
                         p.a_map = amap;
                         p.b_map = bmap;
+                        p.a_map_t = amap_t;
+                        p.b_map_t = bmap_t;
+                        p.a_sym = a_sym ? 1 : 0;
+                        p.b_sym = b_sym ? 1 : 0;
                         p.a_z = static_cast<int>(z);
                         p.b_z = static_cast<int>(z);
                         p.a_mn = A.mn ? 1 : 0;
                         p.b_mn = B.mn ? 1 : 0;
                         p.fmt = g.dt[A.buf] == DT_F16 ? 0 : 1;
                         p.ep = ep;
+                        p.ep.sym = 0;  // upper tiles only (tile list below), no mirrored stores
                         const unsigned pi = static_cast<unsigned>(tprobs.size());
                         tprobs.push_back(p);
                         const int tm = (M + tile_m - 1) / tile_m, tn = (N + tile_n - 1) / tile_n;
@@ -743,7 +755,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
             lr.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
             lr.tc.bad = d_bad;
             lr.tc.status = status;
-            lr.grid = std::min(lr.tc.ntiles, num_sms);
+            // CTA pairs: one cluster of 2 per tile, at most one CTA per SM
+            lr.grid = 2 * std::max(1, std::min(lr.tc.ntiles, num_sms / 2));
         }
         total_flops += lr.flops;
         launches.push_back(lr);

@@ -191,3 +191,53 @@ def test_gpt2_set_full_parity():
         # the update is recovered from an fp32 difference: allow its rounding
         assert e <= TOL_BF16_RELF + 2e-3, (i, w.shapes[i], e)
     print("gpt2 worst relF", worst)
+
+
+def _sigma_maxdiff_gram(a, b):
+    """Largest singular-value difference via the eigenvalues of the short-side
+    Gram matrices (the same singular values as an SVD, at a fraction of its cost)."""
+    def sv(x):
+        x = np.asarray(x, dtype=np.float64)
+        g = x @ x.T if x.shape[0] <= x.shape[1] else x.T @ x
+        return np.sqrt(np.clip(np.linalg.eigvalsh(g), 0, None))
+    return float(np.max(np.abs(sv(a) - sv(b))))
+
+
+def _full_size_sampled(wid, sample, lr=0.01):
+    w = wl.WORKLOADS[wid]
+    W = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=DEV) for i in range(w.count)]
+    G = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=DEV) for i in range(w.count)]
+    M = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=DEV) for i in range(w.count)]
+    keep = {i: (to64(W[i]), to64(G[i]), to64(M[i])) for i in sample}
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=lr)
+    torch.cuda.synchronize()
+    got = {i: to64(W[i]) for i in sample}
+    del W, G, M
+    mo.muon_release_workspace()
+    torch.cuda.empty_cache()
+    for i in sample:
+        W0, G0, M0 = keep[i]
+        r, c = w.shapes[i]
+        n, m = min(r, c), max(r, c)
+        fm = "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
+        _, _, O = orc.muon_step(W0, G0, M0, 0.95, True, lr, form=fm)
+        O_gpu = (W0 - got[i]) / lr
+        e = relF(O_gpu, O)
+        s = _sigma_maxdiff_gram(O_gpu, O)
+        print(w.name, i, w.shapes[i], fm, "relF", e, "max|dsigma|", s)
+        assert e <= TOL_BF16_RELF, (i, w.shapes[i], e)
+        assert s <= TOL_SIGMA, (i, w.shapes[i], s)
+
+
+@pytest.mark.slow
+def test_moe_set_full_size_sampled():
+    """Workload 4 (64 experts, 128 matrices, 1.88 G elements) at full size:
+    first and last matrix of each shape against the oracle."""
+    _full_size_sampled(4, [0, 1, 126, 127])
+
+
+@pytest.mark.slow
+def test_llama8b_set_full_size_sampled():
+    """Workload 5 (Llama-8B Muon set, 224 matrices, 6.98 G elements) at full
+    size: one matrix of each of the four shapes against the oracle."""
+    _full_size_sampled(5, [0, 2, 4, 6])

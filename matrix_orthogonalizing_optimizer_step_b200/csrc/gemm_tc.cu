@@ -24,6 +24,12 @@
 // block through the transposed tensor map of the mirrored upper tile, so no
 // transposed (mirror) store is ever issued.
 //
+// The whole Newton-Schulz chain of a step can run as ONE launch: tiles of all
+// chain slots are listed slot by slot and a tile first waits (bounded) until
+// every tile of the earlier slots of its matrix has been stored, counted in a
+// per-matrix completion counter; matrices progress independently, so the
+// dependency waits of one matrix are filled with other matrices' tiles.
+//
 // Every wait is bounded: on expiry the kernel records a timeout in the device
 // status word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -78,14 +84,25 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     uint32_t issued = 0;
     bool ok = true;
     int last_a = -1, last_b = -1;
+    unsigned seen_mat = ~0u, seen_done = 0;  // counters only grow within a launch
     for (int t = pair; t < L.ntiles && ok; t += npairs) {
-        const uint2 tile = L.tiles[t];
+        const TcTile tile = L.tiles[t];
+        // operands produced by earlier chain slots of the same matrix
+        if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
+            if (!wait_counter(L.done + tile.mat, tile.need, abort_flag)) {
+                ok = false;
+                break;
+            }
+            seen_mat = tile.mat;
+            seen_done = tile.need;
+            fence_proxy_async_global();  // TMA reads see the producers' stores
+        }
         // register copies: the asm statements below clobber memory, so fields
         // read through the problem table would be reloaded inside the K loop
-        const TcProblem& Pg = L.problems[tile.x];
+        const TcProblem& Pg = L.problems[tile.problem];
         const int a_z = Pg.a_z, b_z = Pg.b_z, K = Pg.K;
         const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, a_sym = Pg.a_sym, b_sym = Pg.b_sym;
-        const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
+        const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         const CUtensorMap* ma = L.maps + Pg.a_map;
         const CUtensorMap* mb = L.maps + Pg.b_map;
         const CUtensorMap* ma_t = a_sym ? L.maps + Pg.a_map_t : ma;
@@ -163,11 +180,11 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     bool issued_any = false;
     const uint32_t tiles_base = smem_u32(tiles_smem);
     for (int t = pair; t < L.ntiles && ok; t += npairs) {
-        const uint2 tile = L.tiles[t];
-        const TcProblem& Pg = L.problems[tile.x];
+        const TcTile tile = L.tiles[t];
+        const TcProblem& Pg = L.problems[tile.problem];
         const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, K = Pg.K, fmt = Pg.fmt;  // registers (see producer)
         const int a_sym = Pg.a_sym, b_sym = Pg.b_sym;
-        const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
+        const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         const int nk = (K + BK - 1) / BK;
         if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag)) {
             ok = false;
@@ -230,14 +247,22 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
                                        map_to_cta(smem_u32(&sh->tempty[1]), 0)};
     int acc = 0;
     uint32_t acc_phase = 0;
+    unsigned seen_mat = ~0u, seen_done = 0;
     for (int t = pair; t < L.ntiles; t += npairs) {
-        const uint2 tile = L.tiles[t];
+        const TcTile tile = L.tiles[t];
         // Local copies: the epilogue stores to global memory, so fields read
         // through a reference into the problem table would be reloaded after
         // every store (the compiler cannot rule out aliasing).
-        const Epilogue ep = L.problems[tile.x].ep;
-        const int PM = L.problems[tile.x].M, PN = L.problems[tile.x].N;
-        const int bi = static_cast<int>(tile.y >> 16), bj = static_cast<int>(tile.y & 0xFFFFu);
+        const Epilogue ep = L.problems[tile.problem].ep;
+        const int PM = L.problems[tile.problem].M, PN = L.problems[tile.problem].N;
+        const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
+        // the epilogue inputs (C1) come from earlier slots: acquire them too
+        if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
+            if (lane == 0) (void)wait_counter(L.done + tile.mat, tile.need, abort_flag);
+            __syncwarp();
+            seen_mat = tile.mat;
+            seen_done = tile.need;
+        }
         const bool skip = ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0;
         const float sig = ep.sigma ? *ep.sigma : 1.f;
         const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;
@@ -270,6 +295,11 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
             }
         }
         tc_fence_before();
+        if (L.done) {
+            // this warp's stores are visible before the tile counts as done
+            __syncwarp();
+            if (lane == 0) red_release_add_gpu(L.done + tile.mat, 1u);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
         if (++acc == 2) {
@@ -335,6 +365,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 size_t gemm_tc_smem_bytes() { return SMEM_BYTES; }
 int gemm_tc_tile_m() { return BMP; }
 int gemm_tc_tile_n() { return BN; }
+
+// CTA pairs that can be resident at once (the chained launch needs all of its
+// pairs co-resident: a tile may wait for tiles of any other pair).
+int gemm_tc_max_pairs() {
+    static int cached = -1;
+    if (cached >= 0) return cached;
+    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    cached = n;
+    return n;
+}
 
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream) {
     static bool configured = false;

@@ -7,18 +7,33 @@
 
 namespace muon {
 
+// One tile of work.  Tiles of a matrix's later chain slots depend on all of
+// its earlier tiles: before fetching operands, a tile waits until
+// done[mat] >= need (done counts epilogue-warp completions, 2 CTAs x 8 warps
+// per tile).  need = 0 means no dependency (one launch per chain slot).
+struct TcTile {
+    unsigned problem;
+    unsigned bibj;  // (tile_row << 16) | tile_col
+    unsigned mat;   // matrix index (completion counter)
+    unsigned need;
+};
+
 struct TcLaunch {
     const TcProblem* problems;
-    const uint2* tiles;  // {problem index, (tile_row << 16) | tile_col}
+    const TcTile* tiles;
     int ntiles;
     const CUtensorMap* maps;
     const int* bad;       // per-matrix non-finite flags
+    unsigned* done;       // per-matrix completion counters (zeroed before the launch), or null
     DeviceStatus* status;
 };
+
+constexpr unsigned kTileArrivals = 16;  // epilogue warps of a CTA pair
 
 size_t gemm_tc_smem_bytes();
 int gemm_tc_tile_m();
 int gemm_tc_tile_n();
+int gemm_tc_max_pairs();
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream);
 
 struct F32Launch {
@@ -47,6 +62,8 @@ struct MomLaunch {
     int* bad;           // per matrix non-finite flag
     DeviceStatus* status;
     int mat_index_base; // index of mats[0] in the caller's numbering (status reporting)
+    unsigned* done;     // GEMM completion counters to zero for the next chain launch (or null)
+    int ndone;
 };
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream);
 

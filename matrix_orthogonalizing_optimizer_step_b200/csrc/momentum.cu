@@ -86,6 +86,8 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     __shared__ double red_d[kThreads / 32];
     __shared__ int is_last;
     const long long chunk = blockIdx.x;
+    if (chunk == 0 && L.done)  // the chained GEMM that follows counts tile completions from zero
+        for (int i = threadIdx.x; i < L.ndone; i += kThreads) L.done[i] = 0u;
     const int mi = find_matrix(L.nmats, chunk, L.mats);
     const MomMatrix Mx = L.mats[mi];  // local copy: no reloads after global stores
     const long long numel = Mx.rows * Mx.cols;

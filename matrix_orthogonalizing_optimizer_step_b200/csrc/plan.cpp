@@ -20,6 +20,7 @@
 #include "plan.h"
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <tuple>
@@ -452,6 +453,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     const size_t off_counters = take(sizeof(int) * nm);
     const size_t off_scale = take(sizeof(float) * 4 * nm);
     const size_t off_bad = take(sizeof(int) * nm);
+    const size_t off_done = take(sizeof(unsigned) * nm);
     const size_t off_moms = take(sizeof(MomMatrix) * nm);
     const size_t off_smats = take(sizeof(ScaleMatrix) * nm);
 
@@ -475,7 +477,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                                   g.mats.size();
                 }
     }
-    const size_t off_tiles = take(sizeof(uint2) * std::max<size_t>(ntiles_max, 1));
+    const size_t off_tiles = take(sizeof(TcTile) * std::max<size_t>(ntiles_max, 1));
     // tensor maps: at most 2 operands per op per group, each with a transposed
     // map when symmetric (deduplicated below)
     size_t nmaps_max = 0;
@@ -501,6 +503,34 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     int* d_counters = reinterpret_cast<int*>(base + off_counters);
     float* d_scale = reinterpret_cast<float*>(base + off_scale);
     int* d_bad = reinterpret_cast<int*>(base + off_bad);
+    unsigned* d_done = reinterpret_cast<unsigned*>(base + off_done);
+    // One chained launch for the whole tensor-core chain (tiles wait on
+    // per-matrix completion counters), unless per-slot launches are asked for
+    // (per-op tracing) or the co-resident pair count is unknown.
+    // Chaining pays where slots are short (few tile rounds per CTA pair, so
+    // launch fill and drain dominate); long slots keep one launch per slot.
+    // MUON_CHAIN_LAUNCH=1 / MUON_SLOT_LAUNCHES=1 force either mode.
+    const int max_pairs = f32 ? 0 : gemm_tc_max_pairs();
+    bool chained = false;
+    if (!f32 && max_pairs > 0) {
+        size_t ntiles_est = 0, nslots_est = 0;
+        for (const Group& g : groups) {
+            nslots_est = std::max(nslots_est, g.slots.size());
+            for (const Slot& sl : g.slots)
+                for (const OpDesc& op : sl) {
+                    int M, N, K;
+                    OperandGeom A, B;
+                    op_geometry(g, op, M, N, K, A, B);
+                    const size_t tm = (M + tile_m - 1) / tile_m, tn = (N + tile_n - 1) / tile_n;
+                    ntiles_est += (op.sym ? (tm * (tm + 1)) / 2 : tm * tn) * g.mats.size();
+                }
+        }
+        const double rounds_per_slot =
+            nslots_est ? static_cast<double>(ntiles_est) / nslots_est / max_pairs : 0.0;
+        chained = rounds_per_slot < 16.0;
+        if (std::getenv("MUON_CHAIN_LAUNCH")) chained = true;
+        if (std::getenv("MUON_SLOT_LAUNCHES")) chained = false;
+    }
     auto buf_ptr = [&](const Group& g, int b, int z) -> char* {
         return base + g.off[b] + static_cast<size_t>(g.bstride[b]) * z;
     };
@@ -540,6 +570,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         L.bad = d_bad;
         L.status = status;
         L.mat_index_base = 0;
+        L.done = chained ? d_done : nullptr;
+        L.ndone = chained ? nm : 0;
         double elems = 0;
         for (int i = 0; i < nm; ++i) elems += static_cast<double>(rq.rows[i]) * rq.cols[i];
         const double per = dtype_size(rq.in_dt) + dtype_size(u_dt) + (rq.is_step ? 2.0 * dtype_size(rq.mom_dt) : 0.0);
@@ -582,7 +614,24 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     // ---- GEMM launches -------------------------------------------------------------
     std::vector<TcProblem> tprobs;
     std::vector<F32Problem> fprobs;
-    std::vector<uint2> tiles;
+    std::vector<TcTile> tiles;
+    std::vector<unsigned> mat_tiles_done(nm, 0);  // tiles of each matrix in earlier slots (chained launch)
+    // chained launch: matrices ordered by decreasing chain FLOPs (ties: index)
+    std::vector<int> mat_rank(nm, 0);
+    {
+        std::vector<std::pair<double, int>> cost(nm);
+        for (int i = 0; i < nm; ++i) {
+            const Group& g = groups[mat_group[i]];
+            cost[i] = {g.slots.empty() ? 0.0 : ns_flops(g.n, g.m, rq.steps, g.form, rq.restart_mask), i};
+        }
+        std::stable_sort(cost.begin(), cost.end(), [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
+            return a.first > b.first;
+        });
+        for (int r = 0; r < nm; ++r) mat_rank[cost[r].second] = r;
+    }
+    LaunchRec chain;
+    chain.kind = LaunchRec::TC;
+    bool chain_open = false;
     std::vector<CUtensorMap> maps;
     std::map<std::tuple<int, int, int>, int> map_index;  // (group, buf, box kind)
     EncodeTiledFn encode = nullptr;
@@ -628,7 +677,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         const size_t prob_begin = f32 ? fprobs.size() : tprobs.size();
         const size_t tile_begin = tiles.size();
         struct TileRef {
-            uint2 t;
+            TcTile t;
             int k;
         };
         std::vector<TileRef> ltiles;
@@ -733,7 +782,12 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                         for (int bi = 0; bi < tm; ++bi)
                             for (int bj = 0; bj < tn; ++bj) {
                                 if (op.sym && bi * tile_m > bj * tile_n + tile_n - 1) continue;
-                                ltiles.push_back({make_uint2(pi, (static_cast<unsigned>(bi) << 16) | bj), K});
+                                TcTile tt;
+                                tt.problem = pi;
+                                tt.bibj = (static_cast<unsigned>(bi) << 16) | static_cast<unsigned>(bj);
+                                tt.mat = static_cast<unsigned>(mi);
+                                tt.need = chained ? kTileArrivals * mat_tiles_done[mi] : 0u;
+                                ltiles.push_back({tt, K});
                             }
                     }
                 }
@@ -746,20 +800,53 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
             lr.f32.max_n = max_n;
             lr.f32.bad = d_bad;
         } else {
-            // longest K first: a simple LPT order for the persistent CTAs
-            std::stable_sort(ltiles.begin(), ltiles.end(), [](const TileRef& x, const TileRef& y) { return x.k > y.k; });
-            for (const TileRef& t : ltiles) tiles.push_back(t.t);
+            if (chained) {
+                // the same matrix order in every slot (largest chain first), so a
+                // matrix's earlier-slot tiles are long finished when its next
+                // slot's tiles come up
+                std::stable_sort(ltiles.begin(), ltiles.end(), [&](const TileRef& x, const TileRef& y) {
+                    return mat_rank[x.t.mat] < mat_rank[y.t.mat];
+                });
+            } else {
+                // longest K first: a simple LPT order for the persistent CTAs
+                std::stable_sort(ltiles.begin(), ltiles.end(),
+                                 [](const TileRef& x, const TileRef& y) { return x.k > y.k; });
+            }
+            for (const TileRef& t : ltiles) {
+                tiles.push_back(t.t);
+                ++mat_tiles_done[t.t.mat];
+            }
+            if (chained) {
+                // append this slot to the single chained launch
+                chain.flops += lr.flops;
+                total_flops += lr.flops;
+                chain_open = true;
+                continue;
+            }
             lr.tc.problems = reinterpret_cast<const TcProblem*>(base + off_probs);
-            lr.tc.tiles = reinterpret_cast<const uint2*>(base + off_tiles) + tile_begin;
+            lr.tc.tiles = reinterpret_cast<const TcTile*>(base + off_tiles) + tile_begin;
             lr.tc.ntiles = static_cast<int>(tiles.size() - tile_begin);
             lr.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
             lr.tc.bad = d_bad;
+            lr.tc.done = nullptr;
             lr.tc.status = status;
             // CTA pairs: one cluster of 2 per tile, at most one CTA per SM
             lr.grid = 2 * std::max(1, std::min(lr.tc.ntiles, num_sms / 2));
         }
         total_flops += lr.flops;
         launches.push_back(lr);
+    }
+    if (chain_open) {
+        chain.tc.problems = reinterpret_cast<const TcProblem*>(base + off_probs);
+        chain.tc.tiles = reinterpret_cast<const TcTile*>(base + off_tiles);
+        chain.tc.ntiles = static_cast<int>(tiles.size());
+        chain.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
+        chain.tc.bad = d_bad;
+        chain.tc.done = d_done;
+        chain.tc.status = status;
+        // every pair must be co-resident: a tile may wait for any other pair's tiles
+        chain.grid = 2 * std::max(1, std::min(chain.tc.ntiles, max_pairs));
+        launches.push_back(chain);
     }
 
     // ---- upload tables -------------------------------------------------------------
@@ -772,9 +859,10 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     if (e == cudaSuccess) e = up(off_smats, smats.data(), sizeof(ScaleMatrix) * smats.size());
     if (e == cudaSuccess && !tprobs.empty()) e = up(off_probs, tprobs.data(), sizeof(TcProblem) * tprobs.size());
     if (e == cudaSuccess && !fprobs.empty()) e = up(off_probs, fprobs.data(), sizeof(F32Problem) * fprobs.size());
-    if (e == cudaSuccess && !tiles.empty()) e = up(off_tiles, tiles.data(), sizeof(uint2) * tiles.size());
+    if (e == cudaSuccess && !tiles.empty()) e = up(off_tiles, tiles.data(), sizeof(TcTile) * tiles.size());
     if (e == cudaSuccess && !maps.empty()) e = up(off_maps, maps.data(), sizeof(CUtensorMap) * maps.size());
     if (e == cudaSuccess) e = cudaMemsetAsync(d_counters, 0, sizeof(int) * nm, stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(d_done, 0, sizeof(unsigned) * nm, stream);
     if (e != cudaSuccess) {
         err = std::string("table upload failed: ") + cudaGetErrorString(e);
         return MUON_ERR_CUDA;

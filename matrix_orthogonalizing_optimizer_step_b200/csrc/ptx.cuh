@@ -89,6 +89,41 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// ---- cross-CTA dependencies ---------------------------------------------------
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Release-add (GPU scope): every memory operation that happens before it,
+// including other warp lanes' stores ordered by a preceding __syncwarp, is
+// visible to a thread that acquires the counter afterwards.
+__device__ __forceinline__ void red_release_add_gpu(unsigned* p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Order this thread's generic-proxy view of global memory before its later
+// async-proxy (TMA) accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *counter >= need (acquire, GPU scope).  Gives up like mbar_wait.
+__device__ __forceinline__ bool wait_counter(const unsigned* counter, unsigned need, volatile int* abort_flag) {
+    if (ld_acquire_gpu(counter) >= need) return true;
+    const unsigned long long t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(counter) >= need) return true;
+        if ((it & 15u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
+}
+
 // ---- TMA ------------------------------------------------------------------
 
 // Tensor maps live in global memory and are written by the host between

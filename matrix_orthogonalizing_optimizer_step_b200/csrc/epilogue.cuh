@@ -128,13 +128,16 @@ __device__ __forceinline__ void prefetch_row32(const Epilogue& ep, int M, int N,
 // Apply the fused epilogue to a 32-column row segment of the accumulator:
 // row `row`, columns col0 .. col0 + 31 of an M x N output.  `sig` is the
 // problem's sigma (already loaded).
+// kFull = false compiles only what the tensor-core epilogue uses (no mirrored
+// symmetric stores, no second output), keeping its hot loop small.
+template <bool kFull = true>
 __device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, int M, int N, long long row, int col0,
                                                float* acc, const Raw32* pre = nullptr) {
     if (row >= M) return;
     const int nvalid = min(32, N - col0);
     if (nvalid <= 0) return;
     // symmetric outputs: only columns >= row are produced here
-    const int jmin = ep.sym ? max(0, static_cast<int>(row - col0)) : 0;
+    const int jmin = (kFull && ep.sym) ? max(0, static_cast<int>(row - col0)) : 0;
     if (jmin >= nvalid) return;
     float t1[32];
     if (ep.c1) {
@@ -171,6 +174,7 @@ __device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, in
         }
     }
     store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, jmin, nvalid, acc);
+    if (!kFull) return;
     if (ep.o2) store_row32(ep.o2, ep.o2_dt, ep.ldo2, row, col0, jmin, nvalid, acc);
     if (ep.sym) {
         // mirrored copy of the strictly-upper part: (col, row)

@@ -291,7 +291,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
                 float v[32];
 #pragma unroll
                 for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                epilogue_row32(ep, sig, PM, PN, row, col0, v, &pre[cur]);
+                epilogue_row32<false>(ep, sig, PM, PN, row, col0, v, &pre[cur]);
             }
         }
         tc_fence_before();

@@ -5,6 +5,7 @@ from .muon_oracle import (  # noqa: F401
     DEFAULT_EPS,
     DEFAULT_RESTARTS,
     TUNED_COEFFS,
+    adamw_step,
     frobenius_normalize,
     momentum_update,
     muon_step,

@@ -179,3 +179,30 @@ def ns_flops(n, m, steps=5, form="standard", restarts=DEFAULT_RESTARTS):
             if k < e - 1:
                 total += 2 * n ** 3
     return total
+
+
+def adamw_step(p, g, m, v, step, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8,
+               weight_decay=0.1):
+    """One AdamW step for a parameter that Muon does not handle (embeddings,
+    output head, 1-D parameters: [NanoGPT-Muon] "从 SGD 到 Muon" and
+    "工程复现清单", lr 6e-4, betas (0.9, 0.95), weight decay 0.1).
+
+    Decoupled weight decay, then the bias-corrected Adam update, in the
+    plainest reading of AdamW:
+        p <- p - lr * wd * p
+        m <- beta1 m + (1 - beta1) g
+        v <- beta2 v + (1 - beta2) g^2
+        p <- p - lr * (m / (1 - beta1^t)) / (sqrt(v / (1 - beta2^t)) + eps)
+    `step` is t >= 1 (the step being taken).  Returns (p, m, v).
+    """
+    p = np.asarray(p, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    m = np.asarray(m, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    p = p - lr * weight_decay * p
+    m = beta1 * m + (1.0 - beta1) * g
+    v = beta2 * v + (1.0 - beta2) * g * g
+    mhat = m / (1.0 - beta1 ** step)
+    vhat = v / (1.0 - beta2 ** step)
+    p = p - lr * mhat / (np.sqrt(vhat) + eps)
+    return p, m, v

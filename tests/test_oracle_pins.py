@@ -280,3 +280,42 @@ def test_planted_gram_mistakes_are_caught(mutant):
     X /= np.linalg.norm(X)
     std = orc.ns_standard(X, orc.TUNED_COEFFS, 5)
     assert _relF(mutant(X, orc.TUNED_COEFFS, 5), std) > 1e-4
+
+
+# ---------------------------------------------------------------------------
+# AdamW lane
+
+def test_adamw_matches_torch_adamw_fp64():
+    """Against the library routine torch.optim.AdamW (fp64, CPU) over several
+    steps with a changing gradient."""
+    import torch
+    r = _rng(20)
+    p0 = r.standard_normal((7, 13))
+    grads = [r.standard_normal((7, 13)) for _ in range(6)]
+    tp = torch.nn.Parameter(torch.tensor(p0, dtype=torch.float64))
+    opt = torch.optim.AdamW([tp], lr=6e-4, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.1)
+    p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+    for t, g in enumerate(grads, start=1):
+        tp.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        p, m, v = orc.adamw_step(p, g, m, v, t)
+        assert np.allclose(p, tp.detach().numpy(), rtol=1e-13, atol=1e-15)
+
+
+def test_adamw_closed_forms():
+    # constant gradient from zero state: bias-corrected m = g, v = g^2, so the
+    # Adam part of every step is lr * g / (|g| + eps)
+    g = np.array([[0.5, -2.0, 1e-3]])
+    p = np.array([[1.0, 1.0, 1.0]])
+    m = v = np.zeros_like(g)
+    lr, wd = 1e-2, 0.0
+    for t in range(1, 5):
+        p_prev = p
+        p, m, v = orc.adamw_step(p, g, m, v, t, lr=lr, weight_decay=wd)
+        assert np.allclose(p_prev - p, lr * g / (np.abs(g) + 1e-8), rtol=1e-12)
+    # zero gradient: pure decoupled decay, p_t = p_0 (1 - lr wd)^t
+    p0 = np.array([[2.0, -3.0]])
+    p, m, v = p0, np.zeros_like(p0), np.zeros_like(p0)
+    for t in range(1, 6):
+        p, m, v = orc.adamw_step(p, np.zeros_like(p0), m, v, t, lr=0.1, weight_decay=0.2)
+        assert np.allclose(p, p0 * (1 - 0.1 * 0.2) ** t, rtol=1e-14)

@@ -146,6 +146,28 @@ MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* c
 MUON_API int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
               float lr, const int* shape_list, int count);
 
+/*
+ * muon_adamw_step -- AdamW step of the parameters Muon does not handle
+ * (embeddings, output head, 1-D parameters), the other lane of the hybrid
+ * optimizer: [NanoGPT-Muon] "从 SGD 到 Muon" (AdamW for embedding and
+ * classification head and for scalar/vector parameters) and "工程复现清单"
+ * (lr 6e-4, betas (0.9, 0.95), weight decay 0.1).  Per element, in fp32:
+ *     p <- p (1 - lr wd);  m <- beta1 m + (1 - beta1) g;  v <- beta2 v + (1 - beta2) g^2
+ *     p <- p - lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ * params      host array of count device pointers, installed param_dtype, updated in place
+ * grads       host array of count device pointers, bf16, read only
+ * exp_avg     host array of count device pointers, fp32 first moments, updated in place
+ * exp_avg_sq  host array of count device pointers, fp32 second moments, updated in place
+ * numels      host array of count element counts (>= 1); tensors are treated as flat
+ * step        the step being taken (>= 1) for the bias corrections
+ * 0 <= beta1, beta2 < 1; lr, weight_decay, eps finite (eps >= 0).  One grouped
+ * launch on the bound stream; 4-element vector access when every pointer of a
+ * tensor is aligned and its numel is a multiple of 4.
+ */
+MUON_API int muon_adamw_step(void* const* params, const void* const* grads, void* const* exp_avg,
+                             void* const* exp_avg_sq, const long long* numels, int count, float lr, float beta1,
+                             float beta2, float eps, float weight_decay, int step);
+
 /* ---- allocation-free normalisation ---------------------------------------
  *
  * The pages have no counterpart to this call: it exists for callers that
@@ -182,7 +204,7 @@ MUON_API int muon_normalize_noalloc(int batch, int m, int n, const void* X, void
 /* ---- tracing ------------------------------------------------------------ */
 
 typedef struct muon_kernel_stats {
-    char name[32];    /* kernel kind: "momentum_norm", "gemm_tc", "gemm_f32", "scale_apply" */
+    char name[32];    /* kernel kind: "momentum_norm", "gemm_tc", "gemm_f32", "scale_apply", "adamw" */
     long long launches;
     double total_ms;  /* sum of CUDA-event durations on the launching stream */
     double flops;     /* algorithmic FLOPs summed over launches (symmetric products at half cost) */

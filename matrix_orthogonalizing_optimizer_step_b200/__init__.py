@@ -117,6 +117,26 @@ def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
     _check(lib().muon_step(P, G, M, float(mu), 1 if nesterov else 0, float(lr), S, count))
 
 
+def muon_adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
+                    weight_decay=0.1):
+    """AdamW step (the hybrid optimizer's lane for embeddings, head and 1-D
+    parameters) over lists of CUDA tensors, updated in place.  grads are
+    bf16, moments fp32, params the installed config's param dtype."""
+    count = len(params)
+    if not (len(grads) == len(exp_avg) == len(exp_avg_sq) == count) or count == 0:
+        raise ValueError("params, grads, exp_avg and exp_avg_sq must be non-empty lists of equal length")
+    for ts in zip(params, grads, exp_avg, exp_avg_sq):
+        if any(t.numel() != ts[0].numel() or not t.is_contiguous() for t in ts):
+            raise ValueError("each param, grad and moment must be contiguous with one element count")
+    vp = ctypes.c_void_p
+    arr = lambda ts: (vp * count)(*[t.data_ptr() for t in ts])  # noqa: E731
+    N = (ctypes.c_longlong * count)(*[t.numel() for t in params])
+    _bind_stream(params[0].device)
+    _check(lib().muon_adamw_step(arr(params), arr(grads), arr(exp_avg), arr(exp_avg_sq), N, count,
+                                 float(lr), float(betas[0]), float(betas[1]), float(eps),
+                                 float(weight_decay), int(step)))
+
+
 def muon_default_config():
     cfg = _lib.MuonConfig()
     _check(lib().muon_default_config(ctypes.byref(cfg)))

@@ -38,7 +38,7 @@ EXPORTS = (
     "muon_set_stream", "muon_last_error", "muon_release_workspace",
     "muon_device_status", "muon_orthogonalize", "muon_step",
     "muon_profile_enable", "muon_profile_read", "muon_profile_reset",
-    "muon_launch_count", "muon_normalize_noalloc",
+    "muon_launch_count", "muon_normalize_noalloc", "muon_adamw_step",
 )
 
 
@@ -99,6 +99,9 @@ def load(path=LIB_PATH):
         "muon_profile_reset": (c_int, []),
         "muon_launch_count": (ctypes.c_longlong, []),
         "muon_normalize_noalloc": (c_int, [c_int, c_int, c_int, vp, vp, c_int, c_float]),
+        "muon_adamw_step": (c_int, [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                    ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_longlong), c_int,
+                                    c_float, c_float, c_float, c_float, c_float, c_int]),
     }
     assert set(sig) == set(EXPORTS)
     for name, (res, args) in sig.items():

@@ -79,6 +79,26 @@ struct ScaleLaunch {
 };
 cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream);
 
+// AdamW lane: one tensor (flat) of the grouped elementwise launch.
+struct AdamTensor {
+    void* p;          // parameter (fp32 or bf16)
+    const void* g;    // gradient (bf16)
+    float* m;         // first moment (fp32)
+    float* v;         // second moment (fp32)
+    long long numel;
+    long long chunk_begin;
+    int vec_ok;       // numel % 4 == 0 and every pointer aligned for 4-element access
+};
+
+struct AdamLaunch {
+    const AdamTensor* tensors;
+    int ntensors;
+    long long nchunks;
+    int p_dt;
+    float decay, beta1, beta2, lr_c1, c2, eps;
+};
+cudaError_t launch_adamw(const AdamLaunch& L, cudaStream_t stream);
+
 // The stream bound by muon_set_stream, and the message muon_last_error returns.
 cudaStream_t bound_stream();
 void set_last_error(const char* msg);

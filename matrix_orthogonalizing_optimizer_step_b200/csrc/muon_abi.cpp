@@ -32,6 +32,9 @@ struct DeviceState {
     int cc_major = 0, cc_minor = 0;
     DeviceStatus* status = nullptr;
     std::unique_ptr<Plan> plan;
+    void* adam_table = nullptr;  // AdamW tensor table
+    size_t adam_cap = 0;
+    std::vector<AdamTensor> adam_last;  // contents of adam_table
 };
 std::deque<DeviceState> g_devs;  // deque: references stay valid on growth
 
@@ -121,12 +124,12 @@ struct Profiler : ProfileSink {
     bool on = false;
     std::vector<Pending> pending;
     std::vector<cudaEvent_t> pool;
-    muon_kernel_stats stats[4];
+    muon_kernel_stats stats[5];
     cudaEvent_t cur = nullptr;
     Profiler() { reset(); }
     void reset() {
-        static const char* names[4] = {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply"};
-        for (int i = 0; i < 4; ++i) {
+        static const char* names[5] = {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply", "adamw"};
+        for (int i = 0; i < 5; ++i) {
             std::memset(&stats[i], 0, sizeof(stats[i]));
             std::strncpy(stats[i].name, names[i], sizeof(stats[i].name) - 1);
         }
@@ -351,6 +354,82 @@ int muon_step(void* const* params, const void* const* grads, void* const* moment
     return run_plan(ds, rq);
 }
 
+int muon_adamw_step(void* const* params, const void* const* grads, void* const* exp_avg, void* const* exp_avg_sq,
+                    const long long* numels, int count, float lr, float beta1, float beta2, float eps,
+                    float weight_decay, int step) {
+    ensure_cfg();
+    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
+    if (!params || !grads || !exp_avg || !exp_avg_sq || !numels)
+        return fail(MUON_ERR_INVALID_ARG, "params, grads, exp_avg, exp_avg_sq and numels must not be NULL");
+    if (step < 1) return fail(MUON_ERR_INVALID_ARG, "step must be >= 1");
+    if (!std::isfinite(lr) || !std::isfinite(weight_decay) || !(eps >= 0.f) || !std::isfinite(eps) ||
+        !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+        return fail(MUON_ERR_INVALID_ARG, "lr, weight_decay, eps finite; 0 <= beta1, beta2 < 1");
+    std::vector<AdamTensor> t(count);
+    long long chunks = 0;
+    const bool pf32 = g_cfg.param_dtype == MUON_DTYPE_F32;
+    for (int i = 0; i < count; ++i) {
+        if (numels[i] < 1) return fail(MUON_ERR_INVALID_ARG, "numels entries must be >= 1");
+        if (!params[i] || !grads[i] || !exp_avg[i] || !exp_avg_sq[i])
+            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/exp_avg/exp_avg_sq");
+        t[i].p = params[i];
+        t[i].g = grads[i];
+        t[i].m = static_cast<float*>(exp_avg[i]);
+        t[i].v = static_cast<float*>(exp_avg_sq[i]);
+        t[i].numel = numels[i];
+        t[i].chunk_begin = chunks;
+        auto al = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+        t[i].vec_ok = numels[i] % 4 == 0 && al(params[i], pf32 ? 16 : 8) && al(grads[i], 8) && al(exp_avg[i], 16) &&
+                      al(exp_avg_sq[i], 16);
+        chunks += (numels[i] + kMomChunk - 1) / kMomChunk;
+    }
+    DeviceState* ds = nullptr;
+    int st = check_device(&ds, false);
+    if (st != MUON_OK) return st;
+    // the tensor table lives in a small device buffer owned by the library;
+    // a previous launch on the bound stream has read it before this upload runs
+    std::vector<AdamTensor>& last = ds->adam_last;
+    const size_t bytes = sizeof(AdamTensor) * t.size();
+    if (ds->adam_cap < bytes) {
+        if (ds->adam_table) {
+            cudaStreamSynchronize(g_stream);
+            cudaFree(ds->adam_table);
+        }
+        ds->adam_table = nullptr;
+        ds->adam_cap = 0;
+        if (cudaMalloc(&ds->adam_table, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(MUON_ERR_NO_MEMORY, "AdamW table allocation failed");
+        }
+        ds->adam_cap = bytes;
+        last.clear();
+    }
+    if (last.size() != t.size() || std::memcmp(last.data(), t.data(), bytes) != 0) {
+        cudaError_t e = cudaMemcpyAsync(ds->adam_table, t.data(), bytes, cudaMemcpyHostToDevice, g_stream);
+        if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table upload failed: ") + cudaGetErrorString(e));
+        last = t;
+    }
+    AdamLaunch L;
+    L.tensors = static_cast<const AdamTensor*>(ds->adam_table);
+    L.ntensors = count;
+    L.nchunks = chunks;
+    L.p_dt = pf32 ? DT_F32 : DT_BF16;
+    L.decay = static_cast<float>(1.0 - static_cast<double>(lr) * weight_decay);
+    L.beta1 = beta1;
+    L.beta2 = beta2;
+    L.lr_c1 = static_cast<float>(static_cast<double>(lr) / (1.0 - std::pow(static_cast<double>(beta1), step)));
+    L.c2 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(beta2), step)));
+    L.eps = eps;
+    if (g_prof.on) g_prof.before(g_stream);
+    cudaError_t e = launch_adamw(L, g_stream);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(e));
+    ++g_launches;
+    double elems = 0;
+    for (const AdamTensor& x : t) elems += static_cast<double>(x.numel);
+    if (g_prof.on) g_prof.after(g_stream, 4, 0.0, elems * (pf32 ? 26.0 : 22.0));
+    return MUON_OK;
+}
+
 int muon_profile_enable(int on) {
     g_prof.on = on != 0;
     return MUON_OK;
@@ -358,9 +437,9 @@ int muon_profile_enable(int on) {
 
 int muon_profile_read(muon_kernel_stats* out, int max, int* count) {
     g_prof.fold();
-    if (count) *count = 4;
+    if (count) *count = 5;
     if (out)
-        for (int i = 0; i < max && i < 4; ++i) out[i] = g_prof.stats[i];
+        for (int i = 0; i < max && i < 5; ++i) out[i] = g_prof.stats[i];
     return MUON_OK;
 }
 

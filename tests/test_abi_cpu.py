@@ -116,6 +116,6 @@ def test_no_device_reports_cuda_error(lib):
 def test_profile_api_without_device(lib):
     mo.muon_profile_reset()
     stats = mo.muon_profile_read()
-    assert set(stats) == {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply"}
+    assert set(stats) == {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply", "adamw"}
     assert all(v["launches"] == 0 for v in stats.values())
     assert mo.muon_launch_count() >= 0

@@ -184,3 +184,21 @@ def test_aspect_sweep_batch16_sampled(shape, form):
     for j in (0, len(idx) - 1):
         ref = orc.orthogonalize(to64(X[j]), orc.TUNED_COEFFS, 5, form)
         _check(to64(Y[j]), ref, TOL_BF16_RELF)
+
+
+def test_fitted_per_shape_schedule():
+    """Per-shape coefficients fitted on the host (ROOT-style adaptive NS) run
+    through the same kernels and match the oracle with those coefficients;
+    the bf16 output is closer to orthogonal than with the fixed set."""
+    from matrix_orthogonalizing_optimizer_step_b200 import coeffs as C
+    sched = C.fit_schedule(384, 1536)
+    X = wl.make_single(384, 1536, 33, "gaussian", DEV, "bf16")
+    errs = {}
+    for name, co in (("fit", sched), ("tuned", mo.TUNED_COEFFS)):
+        for form in ("standard", "gram"):
+            ref = orc.orthogonalize(to64(X), co, 5, form)
+            Y = _ortho_gpu(X, form, coeffs=co)
+            _check(to64(Y), ref, TOL_BF16_RELF)
+            errs[name, form] = np.mean((np.linalg.svd(to64(Y), compute_uv=False) - 1) ** 2)
+    for form in ("standard", "gram"):
+        assert errs["fit", form] < 0.5 * errs["tuned", form], errs

@@ -47,8 +47,10 @@ def test_adamw_matches_oracle(par_dt):
                for (p, m, v), g in zip(ref, G)]
         for i, (p, m, v) in enumerate(ref):
             gm, gv = to64(M[i]), to64(V[i])
-            assert np.allclose(gm, m, rtol=1e-5, atol=1e-12), i
-            assert np.allclose(gv, v, rtol=1e-5, atol=1e-15), i
+            # fp32 rounding of the terms (beta m and (1 - beta) g) bounds the
+            # error where they cancel: scale by the tensor's magnitude
+            assert np.max(np.abs(gm - m)) <= 1e-6 * np.max(np.abs(m)), i
+            assert np.max(np.abs(gv - v)) <= 1e-6 * np.max(np.abs(v)), i
             gp = to64(P[i])
             if par_dt == "f32":
                 assert np.max(np.abs(gp - p)) <= 1e-6 * lr + 2e-7 * np.max(np.abs(p)), i

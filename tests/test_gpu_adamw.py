@@ -55,9 +55,9 @@ def test_adamw_matches_oracle(par_dt):
             if par_dt == "f32":
                 assert np.max(np.abs(gp - p)) <= 1e-6 * lr + 2e-7 * np.max(np.abs(p)), i
             else:
-                # the GPU stores a bf16 parameter after every step: at most one
-                # rounding (2^-9 relative) per step taken so far, plus slack
-                assert np.max(np.abs(gp - p) / np.maximum(np.abs(p), 1e-3)) <= step * 2.0 ** -8, i
+                # the GPU stores a bf16 parameter after every step: one rounding
+                # per step so far, each up to 2^-8 relative at a binade's bottom
+                assert np.max(np.abs(gp - p) / np.maximum(np.abs(p), 1e-3)) <= step * 2.0 ** -7, i
 
 
 def test_adamw_zero_gradient_is_pure_decay():

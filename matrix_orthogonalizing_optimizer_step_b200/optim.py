@@ -1,0 +1,97 @@
+"""Hybrid Muon + AdamW optimizer over a model's parameters.
+
+[NanoGPT-Muon] "从 SGD 到 Muon": Muon only handles 2-D parameters (linear
+weights, and convolution kernels once flattened to 2-D); scalar and vector
+parameters stay with AdamW, and AdamW is also used for the embedding and the
+output classification head.  "工程复现清单": AdamW lr 6e-4, betas
+(0.9, 0.95), weight decay 0.1; Muon lr 6e-4, momentum 0.95, Nesterov,
+five Newton-Schulz steps.
+
+This class only keeps the per-parameter state buffers and hands device
+pointers to the library's two fused launches (muon_step for the Muon
+group, muon_adamw_step for the AdamW group); all arithmetic runs in CUDA.
+Gradients must be bf16 (the kernels read bf16 gradients).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import muon_adamw_step, muon_step
+
+_ADAMW_NAME_HINTS = ("embed", "wte", "wpe", "lm_head", "head", "classifier")
+
+
+def split_params(named_params):
+    """(muon, adamw) lists of (name, parameter) by the page's rule: Muon for
+    parameters of >= 2 dimensions that are not an embedding or output head,
+    AdamW for everything else."""
+    muon, adamw = [], []
+    for name, p in named_params:
+        if not p.requires_grad:
+            continue
+        lname = name.lower()
+        if p.dim() >= 2 and not any(h in lname for h in _ADAMW_NAME_HINTS):
+            muon.append((name, p))
+        else:
+            adamw.append((name, p))
+    return muon, adamw
+
+
+class MuonHybrid(torch.optim.Optimizer):
+    """Muon for hidden matrices, AdamW for the rest (see module docstring).
+
+    Pass the output of split_params (or two explicit lists of parameters)."""
+
+    def __init__(self, muon_params, adamw_params, lr=6e-4, momentum=0.95, nesterov=True,
+                 adamw_lr=6e-4, adamw_betas=(0.9, 0.95), adamw_eps=1e-8, adamw_weight_decay=0.1):
+        mp = [p for _, p in muon_params] if muon_params and isinstance(muon_params[0], tuple) else list(muon_params)
+        ap = [p for _, p in adamw_params] if adamw_params and isinstance(adamw_params[0], tuple) else list(adamw_params)
+        groups = []
+        if mp:
+            groups.append(dict(params=mp, kind="muon", lr=lr, momentum=momentum, nesterov=nesterov))
+        if ap:
+            groups.append(dict(params=ap, kind="adamw", lr=adamw_lr, betas=adamw_betas, eps=adamw_eps,
+                               weight_decay=adamw_weight_decay))
+        super().__init__(groups, {})
+
+    @torch.no_grad()
+    def step(self, closure=None):
+        loss = closure() if closure is not None else None
+        for g in self.param_groups:
+            ps = [p for p in g["params"] if p.grad is not None]
+            if not ps:
+                continue
+            for p in ps:
+                if p.grad.dtype != torch.bfloat16:
+                    raise TypeError("gradients must be bf16 (the fused kernels read bf16 gradients)")
+            if g["kind"] == "muon":
+                W, G, M = [], [], []
+                for p in ps:
+                    st = self.state[p]
+                    if "momentum" not in st:
+                        st["momentum"] = torch.zeros_like(p, dtype=torch.bfloat16)
+                    # conv kernels and other >2-D weights are flattened to 2-D views
+                    W.append(p.view(p.shape[0], -1))
+                    G.append(p.grad.view(p.shape[0], -1))
+                    M.append(st["momentum"].view(p.shape[0], -1))
+                muon_step(W, G, M, mu=g["momentum"], nesterov=g["nesterov"], lr=g["lr"])
+            else:
+                P, G, M1, M2 = [], [], [], []
+                for p in ps:
+                    st = self.state[p]
+                    if "exp_avg" not in st:
+                        st["exp_avg"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
+                        st["exp_avg_sq"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
+                        st["step"] = 0
+                    st["step"] += 1
+                    P.append(p.view(-1))
+                    G.append(p.grad.view(-1))
+                    M1.append(st["exp_avg"])
+                    M2.append(st["exp_avg_sq"])
+                steps = {self.state[p]["step"] for p in ps}
+                for t in sorted(steps):  # normally one step count for the whole group
+                    idx = [i for i, p in enumerate(ps) if self.state[p]["step"] == t]
+                    muon_adamw_step([P[i] for i in idx], [G[i] for i in idx], [M1[i] for i in idx],
+                                    [M2[i] for i in idx], t, lr=g["lr"], betas=g["betas"], eps=g["eps"],
+                                    weight_decay=g["weight_decay"])
+        return loss

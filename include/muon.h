@@ -79,6 +79,8 @@ typedef struct muon_config {
     float eps;                        /* added to the Frobenius norm (default 1e-7)             */
     int momentum_dtype;               /* MUON_DTYPE_BF16 (default) or MUON_DTYPE_F32            */
     int param_dtype;                  /* MUON_DTYPE_F32 (default) or MUON_DTYPE_BF16            */
+    int grad_dtype;                   /* gradients of muon_step and muon_adamw_step:
+                                         MUON_DTYPE_BF16 (default) or MUON_DTYPE_F32            */
 } muon_config;
 
 /* Library version (MUON_VERSION of the build). */
@@ -135,7 +137,7 @@ MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* c
  *     M <- mu*M + G;  U = G + mu*M (nesterov) or U = M;
  *     O = NS_T(U / (||U||_F + eps));  W <- W - lr*O.
  * params      host array of count device pointers, param_dtype, updated in place
- * grads       host array of count device pointers, bf16, read only
+ * grads       host array of count device pointers, grad_dtype (bf16 default), read only
  * momentum    host array of count device pointers, momentum_dtype, updated in place
  * shape_list  host int[2*count]: rows_i, cols_i of parameter i (>= 1)
  * Coefficients, steps, NS form, restarts, eps and dtypes come from the
@@ -155,7 +157,7 @@ MUON_API int muon_step(void* const* params, const void* const* grads, void* cons
  *     p <- p (1 - lr wd);  m <- beta1 m + (1 - beta1) g;  v <- beta2 v + (1 - beta2) g^2
  *     p <- p - lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
  * params      host array of count device pointers, installed param_dtype, updated in place
- * grads       host array of count device pointers, bf16, read only
+ * grads       host array of count device pointers, installed grad_dtype, read only
  * exp_avg     host array of count device pointers, fp32 first moments, updated in place
  * exp_avg_sq  host array of count device pointers, fp32 second moments, updated in place
  * numels      host array of count element counts (>= 1); tensors are treated as flat

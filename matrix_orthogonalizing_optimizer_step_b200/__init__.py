@@ -96,7 +96,7 @@ def muon_orthogonalize(X, coeffs=TUNED_COEFFS, steps=5, mode="auto", fp32=False)
 def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
     """One Muon step over lists of 2D CUDA tensors (updated in place).
 
-    grads are bf16; momentum and params use the installed config's dtypes.
+    grads, momentum and params use the installed config's dtypes.
     """
     count = len(params)
     if not (len(grads) == len(momentum) == count) or count == 0:
@@ -120,8 +120,8 @@ def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
 def muon_adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
                     weight_decay=0.1):
     """AdamW step (the hybrid optimizer's lane for embeddings, head and 1-D
-    parameters) over lists of CUDA tensors, updated in place.  grads are
-    bf16, moments fp32, params the installed config's param dtype."""
+    parameters) over lists of CUDA tensors, updated in place.  Moments are
+    fp32; params and grads use the installed config's dtypes."""
     count = len(params)
     if not (len(grads) == len(exp_avg) == len(exp_avg_sq) == count) or count == 0:
         raise ValueError("params, grads, exp_avg and exp_avg_sq must be non-empty lists of equal length")
@@ -149,6 +149,7 @@ def _cfg_to_dict(cfg):
         "coeffs": [tuple(cfg.coeffs[3 * k:3 * k + 3]) for k in range(cfg.steps)],
         "mode": cfg.mode, "restart_mask": cfg.restart_mask, "eps": cfg.eps,
         "momentum_dtype": cfg.momentum_dtype, "param_dtype": cfg.param_dtype,
+        "grad_dtype": cfg.grad_dtype,
     }
 
 
@@ -159,7 +160,7 @@ def muon_get_config():
 
 
 def muon_set_config(steps=None, coeffs=None, mode=None, restart_mask=None,
-                    eps=None, momentum_dtype=None, param_dtype=None):
+                    eps=None, momentum_dtype=None, param_dtype=None, grad_dtype=None):
     """Install a config; unspecified fields keep their current values."""
     cfg = _lib.MuonConfig()
     _check(lib().muon_get_config(ctypes.byref(cfg)))
@@ -179,6 +180,8 @@ def muon_set_config(steps=None, coeffs=None, mode=None, restart_mask=None,
         cfg.momentum_dtype = momentum_dtype
     if param_dtype is not None:
         cfg.param_dtype = param_dtype
+    if grad_dtype is not None:
+        cfg.grad_dtype = grad_dtype
     _check(lib().muon_set_config(ctypes.byref(cfg)))
 
 

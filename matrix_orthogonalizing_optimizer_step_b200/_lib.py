@@ -51,6 +51,7 @@ class MuonConfig(ctypes.Structure):
         ("eps", ctypes.c_float),
         ("momentum_dtype", ctypes.c_int),
         ("param_dtype", ctypes.c_int),
+        ("grad_dtype", ctypes.c_int),
     ]
 
 

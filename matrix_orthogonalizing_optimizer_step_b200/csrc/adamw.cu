@@ -7,7 +7,7 @@
 //     p <- p - lr (m c1) / (sqrt(v c2) + eps),  c1 = 1/(1 - b1^t), c2 = 1/(1 - b2^t)
 // One grouped launch over all tensors: one CTA per chunk of 8192 elements of
 // one tensor, 4-element vector access when aligned.  HBM-bound: 26 bytes per
-// element with fp32 parameters (p, m, v read and written, bf16 g read).
+// element with fp32 parameters and bf16 gradients (p, m, v read and written, g read).
 #include <cuda_bf16.h>
 
 #include "epilogue.cuh"
@@ -45,7 +45,7 @@ __device__ __forceinline__ float adam_elem(float p, float g, float& m, float& v,
     return p - k.lr_c1 * m / (sqrtf(v * k.c2) + k.eps);
 }
 
-template <bool P_F32>
+template <bool P_F32, bool G_F32>
 __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
     const long long chunk = blockIdx.x;
     const AdamTensor T = L.tensors[find_tensor(L.tensors, L.ntensors, chunk)];
@@ -66,7 +66,10 @@ __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
                 const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
                 p[0] = a.x, p[1] = a.y, p[2] = b.x, p[3] = b.y;
             }
-            {
+            if (G_F32) {
+                const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(T.g) + e);
+                g[0] = q.x, g[1] = q.y, g[2] = q.z, g[3] = q.w;
+            } else {
                 const uint2 q = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(T.g) + e);
                 const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
                 const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
@@ -95,7 +98,7 @@ __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
             const long long e = e0 + i;
             if (e >= T.numel) break;
             float m = T.m[e], v = T.v[e];
-            const float p = adam_elem(ld_elem(T.p, pdt, e), ld_elem(T.g, DT_BF16, e), m, v, k);
+            const float p = adam_elem(ld_elem(T.p, pdt, e), ld_elem(T.g, G_F32 ? DT_F32 : DT_BF16, e), m, v, k);
             T.m[e] = m;
             T.v[e] = v;
             st_elem(T.p, pdt, e, p);
@@ -108,10 +111,15 @@ __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
 cudaError_t launch_adamw(const AdamLaunch& L, cudaStream_t stream) {
     if (L.nchunks <= 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(L.nchunks));
-    if (L.p_dt == DT_F32)
-        adamw_kernel<true><<<grid, kThreads, 0, stream>>>(L);
+    const bool pf = L.p_dt == DT_F32, gf = L.g_dt == DT_F32;
+    if (pf && gf)
+        adamw_kernel<true, true><<<grid, kThreads, 0, stream>>>(L);
+    else if (pf)
+        adamw_kernel<true, false><<<grid, kThreads, 0, stream>>>(L);
+    else if (gf)
+        adamw_kernel<false, true><<<grid, kThreads, 0, stream>>>(L);
     else
-        adamw_kernel<false><<<grid, kThreads, 0, stream>>>(L);
+        adamw_kernel<false, false><<<grid, kThreads, 0, stream>>>(L);
     return cudaGetLastError();
 }
 

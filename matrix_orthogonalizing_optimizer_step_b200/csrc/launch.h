@@ -82,7 +82,7 @@ cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream);
 // AdamW lane: one tensor (flat) of the grouped elementwise launch.
 struct AdamTensor {
     void* p;          // parameter (fp32 or bf16)
-    const void* g;    // gradient (bf16)
+    const void* g;    // gradient (bf16 or fp32)
     float* m;         // first moment (fp32)
     float* v;         // second moment (fp32)
     long long numel;
@@ -94,7 +94,7 @@ struct AdamLaunch {
     const AdamTensor* tensors;
     int ntensors;
     long long nchunks;
-    int p_dt;
+    int p_dt, g_dt;
     float decay, beta1, beta2, lr_c1, c2, eps;
 };
 cudaError_t launch_adamw(const AdamLaunch& L, cudaStream_t stream);

@@ -207,11 +207,18 @@ cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream) {
         else
             return cudaErrorInvalidValue;
     } else {
-        if (gf || uf) return cudaErrorInvalidValue;
-        if (L.mom_dt == DT_F32)
-            momentum_norm_kernel<false, MOM_F32, false><<<grid, kThreads, 0, stream>>>(L);
-        else
-            momentum_norm_kernel<false, MOM_BF16, false><<<grid, kThreads, 0, stream>>>(L);
+        if (uf) return cudaErrorInvalidValue;
+        if (gf) {
+            if (L.mom_dt == DT_F32)
+                momentum_norm_kernel<true, MOM_F32, false><<<grid, kThreads, 0, stream>>>(L);
+            else
+                momentum_norm_kernel<true, MOM_BF16, false><<<grid, kThreads, 0, stream>>>(L);
+        } else {
+            if (L.mom_dt == DT_F32)
+                momentum_norm_kernel<false, MOM_F32, false><<<grid, kThreads, 0, stream>>>(L);
+            else
+                momentum_norm_kernel<false, MOM_BF16, false><<<grid, kThreads, 0, stream>>>(L);
+        }
     }
     return cudaGetLastError();
 }

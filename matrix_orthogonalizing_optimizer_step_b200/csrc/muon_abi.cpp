@@ -60,6 +60,7 @@ void fill_defaults(muon_config* c) {
     c->eps = 1e-7f;
     c->momentum_dtype = MUON_DTYPE_BF16;
     c->param_dtype = MUON_DTYPE_F32;
+    c->grad_dtype = MUON_DTYPE_BF16;
 }
 
 void ensure_cfg() {
@@ -79,6 +80,8 @@ int check_cfg(const muon_config& c) {
         return fail(MUON_ERR_UNSUPPORTED, "config.momentum_dtype must be BF16 or F32");
     if (c.param_dtype != MUON_DTYPE_BF16 && c.param_dtype != MUON_DTYPE_F32)
         return fail(MUON_ERR_UNSUPPORTED, "config.param_dtype must be BF16 or F32");
+    if (c.grad_dtype != MUON_DTYPE_BF16 && c.grad_dtype != MUON_DTYPE_F32)
+        return fail(MUON_ERR_UNSUPPORTED, "config.grad_dtype must be BF16 or F32");
     return MUON_OK;
 }
 
@@ -337,7 +340,7 @@ int muon_step(void* const* params, const void* const* grads, void* const* moment
     DeviceState* ds = nullptr;
     int st = check_device(&ds, true);
     if (st != MUON_OK) return st;
-    rq.in_dt = DT_BF16;
+    rq.in_dt = g_cfg.grad_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
     rq.mom_dt = g_cfg.momentum_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
     rq.out_dt = g_cfg.param_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
     rq.is_step = true;
@@ -368,6 +371,7 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
     std::vector<AdamTensor> t(count);
     long long chunks = 0;
     const bool pf32 = g_cfg.param_dtype == MUON_DTYPE_F32;
+    const bool gf32 = g_cfg.grad_dtype == MUON_DTYPE_F32;
     for (int i = 0; i < count; ++i) {
         if (numels[i] < 1) return fail(MUON_ERR_INVALID_ARG, "numels entries must be >= 1");
         if (!params[i] || !grads[i] || !exp_avg[i] || !exp_avg_sq[i])
@@ -379,8 +383,8 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
         t[i].numel = numels[i];
         t[i].chunk_begin = chunks;
         auto al = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
-        t[i].vec_ok = numels[i] % 4 == 0 && al(params[i], pf32 ? 16 : 8) && al(grads[i], 8) && al(exp_avg[i], 16) &&
-                      al(exp_avg_sq[i], 16);
+        t[i].vec_ok = numels[i] % 4 == 0 && al(params[i], pf32 ? 16 : 8) && al(grads[i], gf32 ? 16 : 8) &&
+                      al(exp_avg[i], 16) && al(exp_avg_sq[i], 16);
         chunks += (numels[i] + kMomChunk - 1) / kMomChunk;
     }
     DeviceState* ds = nullptr;
@@ -414,6 +418,7 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
     L.ntensors = count;
     L.nchunks = chunks;
     L.p_dt = pf32 ? DT_F32 : DT_BF16;
+    L.g_dt = gf32 ? DT_F32 : DT_BF16;
     L.decay = static_cast<float>(1.0 - static_cast<double>(lr) * weight_decay);
     L.beta1 = beta1;
     L.beta2 = beta2;
@@ -426,7 +431,7 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
     ++g_launches;
     double elems = 0;
     for (const AdamTensor& x : t) elems += static_cast<double>(x.numel);
-    if (g_prof.on) g_prof.after(g_stream, 4, 0.0, elems * (pf32 ? 26.0 : 22.0));
+    if (g_prof.on) g_prof.after(g_stream, 4, 0.0, elems * ((pf32 ? 8.0 : 4.0) + (gf32 ? 4.0 : 2.0) + 16.0));
     return MUON_OK;
 }
 

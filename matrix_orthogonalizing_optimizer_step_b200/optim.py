@@ -10,13 +10,16 @@ five Newton-Schulz steps.
 This class only keeps the per-parameter state buffers and hands device
 pointers to the library's two fused launches (muon_step for the Muon
 group, muon_adamw_step for the AdamW group); all arithmetic runs in CUDA.
-Gradients must be bf16 (the kernels read bf16 gradients).
+Gradients may be fp32 or bf16 (one type per group); the installed config's
+gradient and parameter dtypes are set to match for each launch.
 """
 from __future__ import annotations
 
 import torch
 
-from . import muon_adamw_step, muon_step
+from . import MUON_DTYPE_BF16, MUON_DTYPE_F32, muon_adamw_step, muon_set_config, muon_step
+
+_CODE = {torch.float32: MUON_DTYPE_F32, torch.bfloat16: MUON_DTYPE_BF16}
 
 _ADAMW_NAME_HINTS = ("embed", "wte", "wpe", "lm_head", "head", "classifier")
 
@@ -61,9 +64,11 @@ class MuonHybrid(torch.optim.Optimizer):
             ps = [p for p in g["params"] if p.grad is not None]
             if not ps:
                 continue
-            for p in ps:
-                if p.grad.dtype != torch.bfloat16:
-                    raise TypeError("gradients must be bf16 (the fused kernels read bf16 gradients)")
+            gdt = {p.grad.dtype for p in ps}
+            pdt = {p.dtype for p in ps}
+            if len(gdt) != 1 or len(pdt) != 1 or not (gdt | pdt) <= set(_CODE):
+                raise TypeError("one gradient dtype and one parameter dtype per group, each fp32 or bf16")
+            muon_set_config(grad_dtype=_CODE[gdt.pop()], param_dtype=_CODE[pdt.pop()])
             if g["kind"] == "muon":
                 W, G, M = [], [], []
                 for p in ps:

@@ -31,15 +31,16 @@ def _state(numels, par_dt, seed):
     return P, M, V
 
 
-@pytest.mark.parametrize("par_dt", ["f32", "bf16"])
-def test_adamw_matches_oracle(par_dt):
-    mo.muon_set_config(param_dtype=mo.MUON_DTYPE_F32 if par_dt == "f32" else mo.MUON_DTYPE_BF16)
+@pytest.mark.parametrize("par_dt,grad_dt", [("f32", "bf16"), ("bf16", "bf16"), ("f32", "f32"), ("bf16", "f32")])
+def test_adamw_matches_oracle(par_dt, grad_dt):
+    mo.muon_set_config(param_dtype=mo.MUON_DTYPE_F32 if par_dt == "f32" else mo.MUON_DTYPE_BF16,
+                       grad_dtype=mo.MUON_DTYPE_F32 if grad_dt == "f32" else mo.MUON_DTYPE_BF16)
     numels = NUMELS if par_dt == "f32" else NUMELS[1:]
     P, M, V = _state(numels, par_dt, 40)
     ref = [(to64(p), np.zeros(p.numel()), np.zeros(p.numel())) for p in P]
     lr, b1, b2, eps, wd = 6e-4, 0.9, 0.95, 1e-8, 0.1
     for step in range(1, 4):
-        G = [wl.make_single(1, n, 1000 * step + i, "student_t3", DEV, "bf16", 0.01).view(-1)
+        G = [wl.make_single(1, n, 1000 * step + i, "student_t3", DEV, grad_dt, 0.01).view(-1)
              for i, n in enumerate(numels)]
         mo.muon_adamw_step(P, G, M, V, step, lr=lr, betas=(b1, b2), eps=eps, weight_decay=wd)
         torch.cuda.synchronize()

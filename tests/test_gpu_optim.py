@@ -30,7 +30,7 @@ def test_hybrid_step_matches_oracle():
     torch.manual_seed(0)
     model = Tiny().to(DEV)
     for i, p in enumerate(model.parameters()):
-        p.grad = wl.make_single(1, p.numel(), 700 + i, "student_t3", DEV, "bf16", 0.01).view(p.shape)
+        p.grad = wl.make_single(1, p.numel(), 700 + i, "student_t3", DEV, "f32", 0.01).view(p.shape)
     muon_p, adamw_p = split_params(model.named_parameters())
     before = {n: to64(p) for n, p in model.named_parameters()}
     grads = {n: to64(p.grad) for n, p in model.named_parameters()}

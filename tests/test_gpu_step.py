@@ -34,18 +34,20 @@ def _expected_momentum(M64, G64, mu, dtype):
     return _bf16_round(m) if dtype == "bf16" else m
 
 
-def _make_set(shapes, seed, mom_dt="bf16", par_dt="f32"):
-    G = [wl.make_single(r, c, seed + 3 * i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+def _make_set(shapes, seed, mom_dt="bf16", par_dt="f32", grad_dt="bf16"):
+    G = [wl.make_single(r, c, seed + 3 * i, "student_t3", DEV, grad_dt, 0.01) for i, (r, c) in enumerate(shapes)]
     M = [wl.make_single(r, c, seed + 3 * i + 1, "student_t3", DEV, mom_dt, 0.01) for i, (r, c) in enumerate(shapes)]
     W = [wl.make_single(r, c, seed + 3 * i + 2, "params", DEV, par_dt) for i, (r, c) in enumerate(shapes)]
     return W, G, M
 
 
-def _run_and_check(shapes, form="auto", mom_dt="bf16", par_dt="f32", nesterov=True, lr=0.1, mu=0.95, seed=1000):
+def _run_and_check(shapes, form="auto", mom_dt="bf16", par_dt="f32", nesterov=True, lr=0.1, mu=0.95, seed=1000,
+                   grad_dt="bf16"):
     mo.muon_set_config(mode=form,
                        momentum_dtype=mo.MUON_DTYPE_F32 if mom_dt == "f32" else mo.MUON_DTYPE_BF16,
-                       param_dtype=mo.MUON_DTYPE_F32 if par_dt == "f32" else mo.MUON_DTYPE_BF16)
-    W, G, M = _make_set(shapes, seed, mom_dt, par_dt)
+                       param_dtype=mo.MUON_DTYPE_F32 if par_dt == "f32" else mo.MUON_DTYPE_BF16,
+                       grad_dtype=mo.MUON_DTYPE_F32 if grad_dt == "f32" else mo.MUON_DTYPE_BF16)
+    W, G, M = _make_set(shapes, seed, mom_dt, par_dt, grad_dt)
     W64, G64, M64 = [to64(t) for t in W], [to64(t) for t in G], [to64(t) for t in M]
     mo.muon_step(W, G, M, mu=mu, nesterov=nesterov, lr=lr)
     torch.cuda.synchronize()
@@ -96,6 +98,11 @@ def test_step_fp32_momentum():
 
 def test_step_bf16_params():
     _run_and_check(SHAPES[:4], par_dt="bf16", lr=0.5)
+
+
+@pytest.mark.parametrize("mom_dt", ["bf16", "f32"])
+def test_step_fp32_gradients(mom_dt):
+    _run_and_check(SHAPES[:4] + [(37, 91)], mom_dt=mom_dt, grad_dt="f32")
 
 
 def test_step_unaligned_columns():

@@ -85,7 +85,7 @@ __device__ __forceinline__ void load_row32(const void* base, int dt, long long l
     for (int j = 0; j < 32; ++j) out[j] = (j < nvalid) ? ld_elem(base, dt, off + j) : 0.f;
 }
 
-// Store columns [jmin, nvalid) of a 32-wide row segment.
+// Store columns [jmin, nvalid) of a 32-wide row segment (one lane's row).
 __device__ __forceinline__ void store_row32(void* base, int dt, long long ld, long long row, int col0, int jmin,
                                             int nvalid, const float* v) {
     const long long off = row * ld + col0;
@@ -125,20 +125,16 @@ __device__ __forceinline__ void prefetch_row32(const Epilogue& ep, int M, int N,
     r.ok = 1;
 }
 
-// Apply the fused epilogue to a 32-column row segment of the accumulator:
-// row `row`, columns col0 .. col0 + 31 of an M x N output.  `sig` is the
-// problem's sigma (already loaded).
-// kFull = false compiles only what the tensor-core epilogue uses (no mirrored
-// symmetric stores, no second output), keeping its hot loop small.
-template <bool kFull = true>
-__device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, int M, int N, long long row, int col0,
-                                               float* acc, const Raw32* pre = nullptr) {
-    if (row >= M) return;
+// The fused epilogue of a 32-column row segment of the accumulator, in place:
+// row `row`, columns col0 .. col0 + 31 of an M x N output become
+// sigma * (alpha * acc + beta * C1) + gamma * C2 + delta * I.  `sig` is the
+// problem's sigma (already loaded).  Rows at or past M are left untouched
+// (returns false); columns past N are computed from zero inputs.
+__device__ __forceinline__ bool epilogue_values32(const Epilogue& ep, float sig, int M, int N, long long row, int col0,
+                                                  float* acc, const Raw32* pre) {
+    if (row >= M) return false;
     const int nvalid = min(32, N - col0);
-    if (nvalid <= 0) return;
-    // symmetric outputs: only columns >= row are produced here
-    const int jmin = (kFull && ep.sym) ? max(0, static_cast<int>(row - col0)) : 0;
-    if (jmin >= nvalid) return;
+    if (nvalid <= 0) return false;
     float t1[32];
     if (ep.c1) {
         if (pre && pre->ok) {
@@ -173,20 +169,7 @@ __device__ __forceinline__ void epilogue_row32(const Epilogue& ep, float sig, in
                 if (j == d) acc[j] += ep.delta;
         }
     }
-    store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, jmin, nvalid, acc);
-    if (!kFull) return;
-    if (ep.o2) store_row32(ep.o2, ep.o2_dt, ep.ldo2, row, col0, jmin, nvalid, acc);
-    if (ep.sym) {
-        // mirrored copy of the strictly-upper part: (col, row)
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const long long col = col0 + j;
-            if (j < nvalid && col > row) {
-                st_elem(ep.o1, ep.o1_dt, col * ep.ldo1 + row, acc[j]);
-                if (ep.o2) st_elem(ep.o2, ep.o2_dt, col * ep.ldo2 + row, acc[j]);
-            }
-        }
-    }
+    return true;
 }
 
 }  // namespace muon

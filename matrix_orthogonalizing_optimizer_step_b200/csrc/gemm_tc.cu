@@ -17,7 +17,10 @@
 //   warp 1      TMEM owner (both CTAs) and MMA issuer (leader only):
 //               two 256-column fp32 accumulators (double-buffered)
 //   warps 2..9  epilogue: tcgen05.ld of 32-column slices, fused combine
-//               sigma*(alpha*acc + beta*C1) + gamma*C2 + delta*I, stores
+//               sigma*(alpha*acc + beta*C1) + gamma*C2 + delta*I; each warp
+//               stages its 32 x 32 result in a 64-byte-swizzled box in
+//               shared memory and one lane stores it with a TMA bulk store
+//               (outputs with an unaligned row pitch: direct stores)
 //
 // Symmetric outputs (X X^T and every product of polynomials in R) are only
 // computed and stored for the upper 256 x 256 tiles; consumers read a lower
@@ -55,7 +58,10 @@ constexpr int EPI_WARPS = 8;
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;  // 2 accumulators x 256 fp32 columns
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int STORE_BOX_BYTES = 64 * 32;  // one TMA store box: 32 rows of 64 bytes
+constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per epilogue warp
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
 
 struct Shared {
     uint64_t full[STAGES];   // leader: both CTAs' operand bytes landed
@@ -71,6 +77,25 @@ struct Shared {
 // kb of the 256-row block `blk` lies in a lower (unstored) tile when blk > kb/4.
 __device__ __forceinline__ bool slice_is_lower(int blk, int kb) { return blk > (kb * BK) / BN; }
 
+// Tile records never change during a launch: read-only path, two 16-byte loads.
+__device__ __forceinline__ TcTile load_tile(const TcTile* tiles, int t) {
+    const uint4* p = reinterpret_cast<const uint4*>(tiles + t);
+    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    TcTile x;
+    x.problem = a.x;
+    x.bibj = a.y;
+    x.mat = a.z;
+    x.need = a.w;
+    x.kf = b.x;
+    x.a_map = static_cast<unsigned short>(b.y & 0xFFFFu);
+    x.b_map = static_cast<unsigned short>(b.y >> 16);
+    x.a_map_t = static_cast<unsigned short>(b.z & 0xFFFFu);
+    x.b_map_t = static_cast<unsigned short>(b.z >> 16);
+    x.a_z = static_cast<unsigned short>(b.w & 0xFFFFu);
+    x.b_z = static_cast<unsigned short>(b.w >> 16);
+    return x;
+}
+
 __device__ __forceinline__ void record_timeout(Shared* sh, DeviceStatus* st) {
     atomicOr(&st->bits, ST_TIMEOUT);
     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
@@ -85,11 +110,20 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     bool ok = true;
     int last_a = -1, last_b = -1;
     unsigned seen_mat = ~0u, seen_done = 0;  // counters only grow within a launch
+    // The next tile's record is fetched while the current tile runs, and its
+    // dependency and tensor maps are acquired right after the current tile's
+    // last fill is issued (the slices still queued in the ring hide the wait),
+    // so consecutive tiles follow each other without a gap in the fills.
+    bool early = false;  // the current tile's dependency was acquired early
+    TcTile nxt;
+    if (pair < L.ntiles) nxt = load_tile(L.tiles, pair);
     for (int t = pair; t < L.ntiles && ok; t += npairs) {
-        const TcTile tile = L.tiles[t];
+        const TcTile tile = nxt;
+        const int tn = t + npairs;
+        if (tn < L.ntiles) nxt = load_tile(L.tiles, tn);
         // operands produced by earlier chain slots of the same matrix
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
-            if (!wait_counter(L.done + tile.mat, tile.need, abort_flag)) {
+            if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag)) {
                 ok = false;
                 break;
             }
@@ -97,25 +131,25 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
             seen_done = tile.need;
             fence_proxy_async_global();  // TMA reads see the producers' stores
         }
-        // register copies: the asm statements below clobber memory, so fields
-        // read through the problem table would be reloaded inside the K loop
-        const TcProblem& Pg = L.problems[tile.problem];
-        const int a_z = Pg.a_z, b_z = Pg.b_z, K = Pg.K;
-        const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, a_sym = Pg.a_sym, b_sym = Pg.b_sym;
+        early = false;
+        const int K = static_cast<int>(tile.kf & kTileMaxK);
+        const unsigned fl = tile.kf >> 24;
+        const bool a_mn = fl & TILE_A_MN, b_mn = fl & TILE_B_MN, a_sym = fl & TILE_A_SYM, b_sym = fl & TILE_B_SYM;
+        const int a_z = tile.a_z, b_z = tile.b_z;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
-        const CUtensorMap* ma = L.maps + Pg.a_map;
-        const CUtensorMap* mb = L.maps + Pg.b_map;
-        const CUtensorMap* ma_t = a_sym ? L.maps + Pg.a_map_t : ma;
-        const CUtensorMap* mb_t = b_sym ? L.maps + Pg.b_map_t : mb;
-        if (Pg.a_map != last_a) {
+        const CUtensorMap* ma = L.maps + tile.a_map;
+        const CUtensorMap* mb = L.maps + tile.b_map;
+        const CUtensorMap* ma_t = a_sym ? L.maps + tile.a_map_t : ma;
+        const CUtensorMap* mb_t = b_sym ? L.maps + tile.b_map_t : mb;
+        if (tile.a_map != last_a) {
             tma_map_acquire(ma);
             if (a_sym) tma_map_acquire(ma_t);
-            last_a = Pg.a_map;
+            last_a = tile.a_map;
         }
-        if (Pg.b_map != last_b) {
+        if (tile.b_map != last_b) {
             tma_map_acquire(mb);
             if (b_sym) tma_map_acquire(mb_t);
-            last_b = Pg.b_map;
+            last_b = tile.b_map;
         }
         const int arow = bi * BMP + static_cast<int>(rank) * BM;   // this CTA's A rows
         const int brow = bj * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows (N)
@@ -153,6 +187,21 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 phase ^= 1u;
             }
         }
+        if (ok && tn < L.ntiles) {
+            if (nxt.need && !(nxt.mat == seen_mat && nxt.need <= seen_done))
+                early = ld_acquire_gpu(L.done + nxt.mat) >= nxt.need;
+            const unsigned nfl = nxt.kf >> 24;
+            if (nxt.a_map != last_a) {
+                tma_map_acquire(L.maps + nxt.a_map);
+                if (nfl & TILE_A_SYM) tma_map_acquire(L.maps + nxt.a_map_t);
+                last_a = nxt.a_map;
+            }
+            if (nxt.b_map != last_b) {
+                tma_map_acquire(L.maps + nxt.b_map);
+                if (nfl & TILE_B_SYM) tma_map_acquire(L.maps + nxt.b_map_t);
+                last_b = nxt.b_map;
+            }
+        }
     }
     if (!ok) record_timeout(sh, L.status);
     // Drain (leader): the last fills of every stage must have landed before
@@ -179,11 +228,16 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     bool ok = true;
     bool issued_any = false;
     const uint32_t tiles_base = smem_u32(tiles_smem);
+    TcTile nxt;
+    if (pair < L.ntiles) nxt = load_tile(L.tiles, pair);
     for (int t = pair; t < L.ntiles && ok; t += npairs) {
-        const TcTile tile = L.tiles[t];
-        const TcProblem& Pg = L.problems[tile.problem];
-        const int a_mn = Pg.a_mn, b_mn = Pg.b_mn, K = Pg.K, fmt = Pg.fmt;  // registers (see producer)
-        const int a_sym = Pg.a_sym, b_sym = Pg.b_sym;
+        const TcTile tile = nxt;
+        if (t + npairs < L.ntiles) nxt = load_tile(L.tiles, t + npairs);  // in flight during this tile
+        const int K = static_cast<int>(tile.kf & kTileMaxK);
+        const unsigned fl = tile.kf >> 24;
+        const int a_mn = (fl & TILE_A_MN) ? 1 : 0, b_mn = (fl & TILE_B_MN) ? 1 : 0;
+        const int a_sym = (fl & TILE_A_SYM) ? 1 : 0, b_sym = (fl & TILE_B_SYM) ? 1 : 0;
+        const int fmt = (fl & TILE_BF16) ? 1 : 0;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         const int nk = (K + BK - 1) / BK;
         if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag)) {
@@ -238,8 +292,8 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     }
 }
 
-__device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base, int warp, int lane, uint32_t rank,
-                               int pair, int npairs) {
+__device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint32_t tmem_base, int warp, int lane,
+                               uint32_t rank, int pair, int npairs) {
     volatile int* abort_flag = &sh->abort;
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // column half of the tile
@@ -248,8 +302,13 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
     int acc = 0;
     uint32_t acc_phase = 0;
     unsigned seen_mat = ~0u, seen_done = 0;
+    uint32_t nstored = 0;  // TMA store boxes issued by this warp (alternating buffers)
+    int last_map = -1;
+    // this lane's 64-byte row of a store box, 16-byte units swizzled (64-byte mode)
+    const uint32_t row_off = static_cast<uint32_t>(lane) * 64;
+    const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
     for (int t = pair; t < L.ntiles; t += npairs) {
-        const TcTile tile = L.tiles[t];
+        const TcTile tile = load_tile(L.tiles, t);
         // Local copies: the epilogue stores to global memory, so fields read
         // through a reference into the problem table would be reloaded after
         // every store (the compiler cannot rule out aliasing).
@@ -265,9 +324,17 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
         }
         const bool skip = ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0;
         const float sig = ep.sigma ? *ep.sigma : 1.f;
-        const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;
+        const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;  // this warp's first row
         const long long row = row0 + lane;
         const int cbase = bj * BN + half * (BN / 2);
+        const bool use_tma = ep.o1_map >= 0;
+        const CUtensorMap* omap = use_tma ? L.maps + ep.o1_map : nullptr;
+        if (use_tma && ep.o1_map != last_map) {
+            if (lane == 0) tma_map_acquire(omap);
+            last_map = ep.o1_map;
+        }
+        const int nbox = ep.o1_dt == DT_F32 ? 2 : 1;  // 64-byte boxes per 32-column slice
+        bool stored = false;
         // prefetch the C1 row segment of the first slice while the MMAs run
         Raw32 pre[2];
         prefetch_row32(ep, PM, PN, row, cbase, pre[0]);
@@ -287,26 +354,66 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t tmem_base
             tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * (BN / 2) + c,
                                r);
             tmem_wait_ld();
-            if (!skip) {
-                float v[32];
+            if (skip || row0 >= PM) continue;  // warp-uniform
+            float v[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-                epilogue_row32<false>(ep, sig, PM, PN, row, col0, v, &pre[cur]);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            const bool valid = epilogue_values32(ep, sig, PM, PN, row, col0, v, &pre[cur]);
+            if (!use_tma) {
+                if (valid) store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, 0, min(32, PN - col0), v);
+                continue;
+            }
+            // staged TMA store: rows past M and columns past N are clipped
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h >= nbox) break;
+                const uint32_t buf = stg + ((nstored & 1u) * STORE_BOX_BYTES);
+                if (lane == 0 && nstored >= 2) bulk_wait_read<1>();  // the box's previous store has read it
+                __syncwarp();
+                if (ep.o1_dt == DT_F32) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float* f = v + 16 * h + 4 * u;
+                        st_shared_v4(buf + row_off + ((static_cast<uint32_t>(u) ^ sw) << 4),
+                                     make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                                                __float_as_uint(f[3])));
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        st_shared_v4(buf + row_off + ((static_cast<uint32_t>(u) ^ sw) << 4), pack8(v + 8 * u, ep.o1_dt));
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(omap, buf, col0 + 16 * h, static_cast<int>(row0), ep.o1_z);
+                    bulk_commit();
+                }
+                ++nstored;
+                stored = true;
             }
         }
+        // the accumulator is free as soon as it has been read
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
         if (L.done) {
-            // this warp's stores are visible before the tile counts as done
+            // this warp's stores are complete and visible before the tile counts as done
+            if (lane == 0 && stored) {
+                bulk_wait_all();
+                fence_proxy_async_global();
+            }
             __syncwarp();
             if (lane == 0) red_release_add_gpu(L.done + tile.mat, 1u);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
         if (++acc == 2) {
             acc = 0;
             acc_phase ^= 1u;
         }
     }
+    // the staging boxes must stay valid until every store has read them
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
@@ -314,7 +421,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem =
         reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    Shared* sh = reinterpret_cast<Shared*>(tiles_smem + STAGES * STAGE_BYTES);
+    uint8_t* store_smem = tiles_smem + STAGES * STAGE_BYTES;  // 1024-byte aligned boxes
+    Shared* sh = reinterpret_cast<Shared*>(store_smem + STORE_BYTES);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_cta_rank();
     const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
@@ -347,7 +455,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base, pair, npairs);
     } else {
-        epilogue_warps(L, sh, tmem_base, warp, lane, rank, pair, npairs);
+        epilogue_warps(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank,
+                       pair, npairs);
     }
 
     tc_fence_before();

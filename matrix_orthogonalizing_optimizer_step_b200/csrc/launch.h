@@ -11,12 +11,23 @@ namespace muon {
 // its earlier tiles: before fetching operands, a tile waits until
 // done[mat] >= need (done counts epilogue-warp completions, 2 CTAs x 8 warps
 // per tile).  need = 0 means no dependency (one launch per chain slot).
+//
+// A tile record also carries everything the TMA producer and the MMA issuer
+// read (K, operand layout flags, tensor maps, batch coordinates): 32 bytes,
+// fetched one tile ahead, so no dependent load of the problem table sits
+// between two tiles of a CTA pair.
 struct TcTile {
-    unsigned problem;
-    unsigned bibj;  // (tile_row << 16) | tile_col
-    unsigned mat;   // matrix index (completion counter)
+    unsigned problem;  // index into the problem table (epilogue, M, N)
+    unsigned bibj;     // (tile_row << 16) | tile_col
+    unsigned mat;      // matrix index (completion counter)
     unsigned need;
+    unsigned kf;       // K (low 24 bits) | operand flags (TILE_*) << 24
+    unsigned short a_map, b_map, a_map_t, b_map_t;  // tensor-map indices (_t: transposed, symmetric operands)
+    unsigned short a_z, b_z;                          // batch coordinates
 };
+static_assert(sizeof(TcTile) == 32, "tile records are loaded as two 16-byte vectors");
+enum { TILE_A_MN = 1, TILE_B_MN = 2, TILE_A_SYM = 4, TILE_B_SYM = 8, TILE_BF16 = 16 };
+constexpr unsigned kTileMaxK = (1u << 24) - 1;
 
 struct TcLaunch {
     const TcProblem* problems;

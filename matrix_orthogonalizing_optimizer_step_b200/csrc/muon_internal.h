@@ -33,6 +33,10 @@ struct Epilogue {
     const void* c2; long long ldc2; int c2_dt;
     void* o1; long long ldo1; int o1_dt;
     void* o2; long long ldo2; int o2_dt;
+    // tensor-core path: TMA store map of o1 (boxes of 64 bytes x 32 rows,
+    // 64-byte swizzle) and the batch coordinate of this problem in it, or
+    // o1_map = -1 (o1 not 16-byte aligned: direct stores)
+    int o1_map, o1_z;
 };
 
 // One tensor-core GEMM problem D[M x N] = A[M x K] * B[K x N] (B given as N x K

@@ -405,6 +405,13 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         mat_z[i] = static_cast<int>(groups[gi].mats.size());
         groups[gi].mats.push_back(i);
     }
+    // tile records hold K in 24 bits and batch coordinates in 16 bits
+    for (const Group& g : groups) {
+        if (!f32 && (static_cast<unsigned>(g.m) > kTileMaxK || g.mats.size() > 65535)) {
+            err = "a shape group exceeds the tensor-core tile limits (K < 2^24, at most 65535 matrices of one shape)";
+            return MUON_ERR_UNSUPPORTED;
+        }
+    }
     for (Group& g : groups) {
         if (rq.steps > 0) {
             if (g.form == FORM_GRAM)
@@ -483,6 +490,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     size_t nmaps_max = 0;
     for (const Group& g : groups)
         for (const Slot& s : g.slots) nmaps_max += 4 * s.size();
+    // TMA store maps: one per workspace buffer of a group, one per caller output
+    nmaps_max += groups.size() * NBUF + static_cast<size_t>(nm);
     const size_t off_maps = take(sizeof(CUtensorMap) * std::max<size_t>(nmaps_max, 1));
     const size_t need = cursor;
 
@@ -639,7 +648,51 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         encode = get_encoder(err);
         if (!encode) return MUON_ERR_CUDA;
     }
-    enum { BOX_KA = 0, BOX_KB = 1, BOX_MN = 2 };
+    enum { BOX_KA = 0, BOX_KB = 1, BOX_MN = 2, BOX_ST = 3 };
+    const bool tma_store = !f32 && !(std::getenv("MUON_TMA_STORE") && std::atoi(std::getenv("MUON_TMA_STORE")) == 0);
+    auto tmap_dtype = [](int dt) {
+        return dt == DT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                            : (dt == DT_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+    };
+    // Store maps: boxes of 64 bytes (32 16-bit or 16 fp32 elements) x 32 rows
+    // with the 64-byte swizzle, the epilogue's staging layout.  -1 when the
+    // buffer breaks the TMA alignment rules (16-byte base and row pitch).
+    auto encode_store_map = [&](void* ptr, int dt, cuuint64_t inner, cuuint64_t outer, cuuint64_t batch,
+                                cuuint64_t ld, cuuint64_t bstride) -> int {
+        const int es = dtype_size(dt);
+        if ((reinterpret_cast<uintptr_t>(ptr) & 15) != 0 || (ld * es) % 16 != 0 || bstride % 16 != 0) return -1;
+        if (maps.size() >= 65535 || maps.size() >= nmaps_max) return -1;
+        cuuint64_t dims[3] = {inner, outer, batch};
+        cuuint64_t strides[2] = {ld * es, bstride};
+        cuuint32_t boxd[3] = {static_cast<cuuint32_t>(64 / es), 32, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        CUtensorMap m;
+        std::memset(&m, 0, sizeof(m));
+        if (encode(&m, tmap_dtype(dt), 3, ptr, dims, strides, boxd, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return -1;
+        maps.push_back(m);
+        return static_cast<int>(maps.size()) - 1;
+    };
+    std::map<std::pair<int, int>, int> store_map_index;  // (group, buffer) or (-1 - matrix, OUTB)
+    auto get_store_map = [&](int gi, int b, int mi) -> int {
+        const auto key = b == OUTB ? std::make_pair(-1 - mi, b) : std::make_pair(gi, b);
+        auto it = store_map_index.find(key);
+        if (it != store_map_index.end()) return it->second;
+        int idx;
+        if (b == OUTB) {
+            const cuuint64_t r = rq.rows[mi], c = rq.cols[mi];
+            idx = encode_store_map(rq.out[mi], rq.out_dt, c, r, 1, c, r * c * dtype_size(rq.out_dt));
+        } else {
+            const Group& g = groups[gi];
+            const bool xb = is_x_buf(b);
+            idx = encode_store_map(base + g.off[b], g.dt[b], xb ? g.cols_w : g.n, xb ? g.rows_w : g.n, g.mats.size(),
+                                   xb ? g.ldx : g.ldn, g.bstride[b]);
+        }
+        store_map_index[key] = idx;
+        return idx;
+    };
     auto get_map = [&](int gi, int b, int box) -> int {
         auto key = std::make_tuple(gi, b, box);
         auto it = map_index.find(key);
@@ -663,6 +716,10 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
             err = "cuTensorMapEncodeTiled failed (" + std::to_string(static_cast<int>(r)) + ")";
+            return -1;
+        }
+        if (maps.size() >= 65535 || maps.size() >= nmaps_max) {
+            err = "too many tensor maps for one plan";
             return -1;
         }
         maps.push_back(m);
@@ -741,6 +798,10 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                     tmp = nullptr;
                     bind(op.o2, tmp, ep.ldo2, ep.o2_dt);
                     ep.o2 = const_cast<void*>(tmp);
+                    ep.o1_map = -1;
+                    ep.o1_z = op.o1 == OUTB ? 0 : static_cast<int>(z);
+                    if (tma_store && op.o1 >= 0)
+                        ep.o1_map = get_store_map(static_cast<int>(gi), op.o1, mi);
                     if (f32) {
                         F32Problem p;
                         std::memset(&p, 0, sizeof(p));
@@ -783,7 +844,19 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                             for (int bj = 0; bj < tn; ++bj) {
                                 if (op.sym && bi * tile_m > bj * tile_n + tile_n - 1) continue;
                                 TcTile tt;
+                                std::memset(&tt, 0, sizeof(tt));
                                 tt.problem = pi;
+                                tt.kf = static_cast<unsigned>(K) |
+                                        static_cast<unsigned>((p.a_mn ? TILE_A_MN : 0) | (p.b_mn ? TILE_B_MN : 0) |
+                                                              (p.a_sym ? TILE_A_SYM : 0) | (p.b_sym ? TILE_B_SYM : 0) |
+                                                              (p.fmt ? TILE_BF16 : 0))
+                                            << 24;
+                                tt.a_map = static_cast<unsigned short>(p.a_map);
+                                tt.b_map = static_cast<unsigned short>(p.b_map);
+                                tt.a_map_t = static_cast<unsigned short>(p.a_sym ? p.a_map_t : 0);
+                                tt.b_map_t = static_cast<unsigned short>(p.b_sym ? p.b_map_t : 0);
+                                tt.a_z = static_cast<unsigned short>(p.a_z);
+                                tt.b_z = static_cast<unsigned short>(p.b_z);
                                 tt.bibj = (static_cast<unsigned>(bi) << 16) | static_cast<unsigned>(bj);
                                 tt.mat = static_cast<unsigned>(mi);
                                 tt.need = chained ? kTileArrivals * mat_tiles_done[mi] : 0u;

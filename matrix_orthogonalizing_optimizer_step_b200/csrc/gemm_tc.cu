@@ -12,7 +12,7 @@
 // than a single-CTA 128 x 256 tile.
 //
 //   warp 0      TMA producer (both CTAs): 64-wide K slices of its halves of A
-//               and B into a 6-stage ring (128-byte swizzle, no multicast);
+//               and B into a 5-stage ring (128-byte swizzle, no multicast);
 //               the transaction bytes of both CTAs land on the leader's barrier
 //   warp 1      TMEM owner (both CTAs) and MMA issuer (leader only):
 //               two 256-column fp32 accumulators (double-buffered)
@@ -50,7 +50,7 @@ constexpr int BMP = 2 * BM;    // rows per CTA pair
 constexpr int BN = 256;        // output columns per tile
 constexpr int BNH = BN / 2;    // B rows (N) loaded per CTA
 constexpr int BK = 64;
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA

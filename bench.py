@@ -217,10 +217,24 @@ def barrier(world, device=None):
             dist.barrier()
 
 
-def traffic_from_profiles(kernel_src):
-    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel source (else None)."""
+def kernel_sources_hash():
+    """sha256 (first 16 hex digits) over every source of libmuon.so: a stored
+    ncu figure is only reported while the kernels it was taken on are unchanged."""
+    import glob
     import hashlib
+    csrc = os.path.join(HERE, "matrix_orthogonalizing_optimizer_step_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(csrc, "*"))):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            h.update(os.path.basename(f).encode())
+            with open(f, "rb") as fh:
+                h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profiles():
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
     p = os.path.join(HERE, "profiles", "gemm_tc_gpt2_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -230,12 +244,7 @@ def traffic_from_profiles(kernel_src):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-    try:
-        with open(kernel_src, "rb") as fh:
-            h = hashlib.sha256(fh.read()).hexdigest()[:16]
-    except OSError:
-        return None
-    if vals.get("kernel_source_sha256_16") != h:
+    if vals.get("kernel_sources_sha256_16") != kernel_sources_hash():
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -334,8 +343,7 @@ def run_ours(args):
     peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     peak_tf = peak_sust if long_step else peak_burst
-    traffic = traffic_from_profiles(os.path.join(HERE, "matrix_orthogonalizing_optimizer_step_b200",
-                                                 "csrc", "gemm_tc.cu"))
+    traffic = traffic_from_profiles()
     roofline = {
         "kernel": "gemm_tc (tcgen05 grouped GEMM, all Newton-Schulz products)",
         "bound": "tensor", "achieved": round(gemm_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",

@@ -319,3 +319,43 @@ def test_adamw_closed_forms():
     for t in range(1, 6):
         p, m, v = orc.adamw_step(p, np.zeros_like(p0), m, v, t, lr=0.1, weight_decay=0.2)
         assert np.allclose(p, p0 * (1 - 0.1 * 0.2) ** t, rtol=1e-14)
+
+
+def _adamw_mutant(kind):
+    """Plausible wrong AdamW variants (planted on the CPU, never in the oracle)."""
+    def step(p, g, m, v, t, lr=6e-4, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.1):
+        if kind == "coupled":
+            g = g + weight_decay * p  # L2 regularisation instead of decoupled decay
+        elif kind != "decay_after":
+            p = p - lr * weight_decay * p
+        m = beta1 * m + (1 - beta1) * g
+        v = beta2 * v + (1 - beta2) * g * g
+        if kind == "no_bias_correction":
+            upd = m / (np.sqrt(v) + eps)
+        else:
+            upd = (m / (1 - beta1 ** t)) / (np.sqrt(v / (1 - beta2 ** t)) + eps)
+        p_new = p - lr * upd
+        if kind == "decay_after":
+            p_new = p_new - lr * weight_decay * p_new
+        return p_new, m, v
+    return step
+
+
+@pytest.mark.parametrize("kind", ["no_bias_correction", "coupled", "decay_after"])
+def test_adamw_pin_rejects_planted_mistakes(kind):
+    """The torch.optim.AdamW comparison above tells each mutant apart."""
+    import torch
+    r = _rng(21)
+    p0 = r.standard_normal((5, 9))
+    grads = [r.standard_normal((5, 9)) for _ in range(4)]
+    tp = torch.nn.Parameter(torch.tensor(p0, dtype=torch.float64))
+    opt = torch.optim.AdamW([tp], lr=1e-2, betas=(0.9, 0.95), eps=1e-8, weight_decay=0.1)
+    step = _adamw_mutant(kind)
+    p, m, v = p0.copy(), np.zeros_like(p0), np.zeros_like(p0)
+    worst = 0.0
+    for t, g in enumerate(grads, start=1):
+        tp.grad = torch.tensor(g, dtype=torch.float64)
+        opt.step()
+        p, m, v = step(p, g, m, v, t, lr=1e-2)
+        worst = max(worst, float(np.max(np.abs(p - tp.detach().numpy()))))
+    assert worst > 1e-7, worst

@@ -30,7 +30,9 @@ Readings where the sources are silent (each listed in the design doc):
 * Frobenius normalisation X0 = U / (||U||_F + eps), eps = 1e-7;
 * the Gram side is the shorter one: a matrix with rows > cols is transposed;
 * update W <- W - lr * O with no extra shape factor and no weight decay;
-* restart schedule: a set of step indices at which X is re-materialised.
+* restart schedule: a set of step indices at which X is re-materialised;
+* soft-threshold split ([ROOT] "ROOT优化器的技术创新"): outliers are the
+  soft-thresholded momentum at lam / 2, the robust part is the rest.
 """
 from __future__ import annotations
 
@@ -141,15 +143,37 @@ def orthogonalize(U, coeffs=TUNED_COEFFS, steps=5, form="standard",
     return O.T if trans else O
 
 
+def soft_threshold_split(M, lam):
+    """Split of a momentum matrix into a robust part and an outlier part
+    ([ROOT] "ROOT优化器的技术创新": soft-threshold denoising, objective
+    min ||M - B - O||_F^2 + lam ||O||_1, only the robust part B is
+    orthogonalised).
+
+    Reading: O is the minimiser of ||M - O||_F^2 + lam ||O||_1, which is
+    elementwise soft-thresholding at lam / 2,
+        O = sign(M) * max(|M| - lam/2, 0),
+    and B = M - O is what remains (M clipped to [-lam/2, lam/2]).
+    Returns (B, O).
+    """
+    M = np.asarray(M, dtype=np.float64)
+    O = np.sign(M) * np.maximum(np.abs(M) - lam / 2.0, 0.0)
+    return M - O, O
+
+
 def muon_step(W, G, M, mu=0.95, nesterov=True, lr=6e-4, coeffs=TUNED_COEFFS,
               steps=5, form="standard", eps=DEFAULT_EPS,
-              restarts=DEFAULT_RESTARTS):
+              restarts=DEFAULT_RESTARTS, soft_threshold=0.0):
     """One Muon step for one 2D parameter ([Gram-NS] "ข้อได้เปรียบของอัลกอริทึม";
     [NanoGPT-Muon] "从 SGD 到 Muon"): momentum, orthogonalise, W <- W - lr * O.
+    With soft_threshold = lam > 0 the matrix orthogonalised is the robust
+    part of U ([ROOT] "ROOT优化器的技术创新", see soft_threshold_split);
+    the momentum buffer keeps the full M.
 
     Returns (W_new, M_new, O).
     """
     M_new, U = momentum_update(M, G, mu, nesterov)
+    if soft_threshold > 0:
+        U, _ = soft_threshold_split(U, soft_threshold)
     O = orthogonalize(U, coeffs, steps, form, eps, restarts)
     W_new = np.asarray(W, dtype=np.float64) - lr * O
     return W_new, M_new, O

@@ -359,3 +359,54 @@ def test_adamw_pin_rejects_planted_mistakes(kind):
         p, m, v = step(p, g, m, v, t, lr=1e-2)
         worst = max(worst, float(np.max(np.abs(p - tp.detach().numpy()))))
     assert worst > 1e-7, worst
+
+
+# ---------------------------------------------------------------------------
+# Soft-threshold split ([ROOT] "ROOT优化器的技术创新")
+
+def test_soft_threshold_split_minimises_the_objective_by_brute_force():
+    """Each element of O minimises (m - o)^2 + lam |o| (the objective with the
+    robust part held at the residual): check against a dense grid search."""
+    r = _rng(30)
+    M = r.standard_normal((4, 6)) * 2.0
+    lam = 1.3
+    _, O = orc.soft_threshold_split(M, lam)
+    grid = np.linspace(-8, 8, 160001)
+    for mval, o in zip(M.ravel(), O.ravel()):
+        f = (mval - grid) ** 2 + lam * np.abs(grid)
+        best = grid[np.argmin(f)]
+        assert abs(best - o) <= 2e-4, (mval, o, best)
+
+
+def test_soft_threshold_split_invariants_and_limits():
+    r = _rng(31)
+    M = r.standard_normal((9, 5))
+    lam = 0.8
+    B, O = orc.soft_threshold_split(M, lam)
+    assert np.allclose(B + O, M, rtol=0, atol=1e-15)        # a split of M
+    assert np.all(np.abs(B) <= lam / 2 + 1e-15)             # robust part bounded
+    small = np.abs(M) <= lam / 2
+    assert np.all(O[small] == 0) and np.all(B[small] == M[small])
+    assert np.all(np.sign(O[~small]) == np.sign(M[~small]))
+    # lam -> infinity: no outliers, plain Muon; lam -> 0: everything is outlier
+    B_inf, O_inf = orc.soft_threshold_split(M, 1e9)
+    assert np.array_equal(B_inf, M) and not O_inf.any()
+    B0, _ = orc.soft_threshold_split(M, 0.0)
+    assert not B0.any()
+
+
+def test_soft_threshold_muon_step_orthogonalises_the_clipped_update():
+    r = _rng(32)
+    G = r.standard_normal((6, 10)) * 0.01
+    G[2, 3] = 3.0  # one outlier
+    W = r.standard_normal((6, 10))
+    M = np.zeros_like(G)
+    lam = 0.06
+    W1, M1, O = orc.muon_step(W, G, M, 0.9, True, 0.1, form="standard", soft_threshold=lam)
+    _, U = orc.momentum_update(M, G, 0.9, True)
+    assert np.allclose(M1, G)  # the momentum buffer keeps the outlier
+    expect = orc.orthogonalize(np.clip(U, -lam / 2, lam / 2), form="standard")
+    assert np.allclose(O, expect, rtol=0, atol=1e-14)
+    # without the split the outlier dominates: the two updates differ
+    _, _, O_plain = orc.muon_step(W, G, M, 0.9, True, 0.1, form="standard")
+    assert np.linalg.norm(O - O_plain) > 0.1

@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--soft-threshold", type=float, default=0.0,
+                    help="lam of the soft-threshold split of the update (0 = plain Muon)")
     ap.add_argument("--subset", type=int, default=0,
                     help="use only the first N matrices of the workload (small profiling cases)")
     return ap.parse_args()
@@ -70,7 +72,7 @@ def _ns_form_for(n, m, form):
     return "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
 
 
-def cpu_oracle_step_ms(w, budget_s, form="auto"):
+def cpu_oracle_step_ms(w, budget_s, form="auto", soft_threshold=0.0):
     """Time the fp64 oracle on a bounded sample of one step of workload w and
     scale to the whole step.  Matrices are taken in order (one of each shape
     first) until the time budget is spent; the per-shape mean time is
@@ -104,7 +106,7 @@ def cpu_oracle_step_ms(w, budget_s, form="auto"):
         if w.full_step:
             M = wl.make_matrix(w, i, wl.ROLE_MOMENTUM).to(torch.float64).numpy()
             W = wl.make_matrix(w, i, wl.ROLE_PARAM).to(torch.float64).numpy()
-            orc.muon_step(W, G, M, 0.95, True, 6e-4, form=fm)
+            orc.muon_step(W, G, M, 0.95, True, 6e-4, form=fm, soft_threshold=soft_threshold)
         else:
             orc.orthogonalize(G, form=fm)
         per_shape.setdefault((r, c), []).append(time.perf_counter() - t0)
@@ -271,7 +273,7 @@ def run_ours(args):
         grads = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev) for i in range(w.count)]
         moms = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
         mo.muon_reset_config()
-        mo.muon_set_config(mode=args.form)
+        mo.muon_set_config(mode=args.form, soft_threshold=args.soft_threshold)
 
         def step():
             mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
@@ -411,7 +413,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, sample = cpu_oracle_step_ms(w, args.cpu_seconds, args.form)
+        v, cores, sample = cpu_oracle_step_ms(w, args.cpu_seconds, args.form, args.soft_threshold)
         cpu = {"value": round(v, 2), "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample}
 
     if rank == 0:
@@ -425,6 +427,7 @@ def run_ours(args):
                        "elements": w.elements, "ns_steps": 5, "ns_form": args.form,
                        "coeffs": [3.4445, -4.775, 2.0315], "momentum": 0.95, "nesterov": True,
                        "lr": 6e-4, "momentum_dtype": w.momentum_dtype, "param_dtype": w.param_dtype,
+                       "soft_threshold": args.soft_threshold,
                        "l2": f"inputs larger than L2: {in_bytes_resident / 1e6:.0f} MB read per step",
                        "parallelism": f"replica x{world} (independent per GPU)"},
             "ns_tflops_per_step": round(ns_tflops, 2),
@@ -446,11 +449,11 @@ def run_reference(args):
     w = wl.WORKLOADS[args.workload]
     budget = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
-        cpu_oracle_step_ms(w, budget, args.form)
+        cpu_oracle_step_ms(w, budget, args.form, args.soft_threshold)
     vals = []
     cores, sample = None, None
     for _ in range(args.steps):
-        v, cores, sample = cpu_oracle_step_ms(w, budget, args.form)
+        v, cores, sample = cpu_oracle_step_ms(w, budget, args.form, args.soft_threshold)
         vals.append(v)
     value = statistics.fmean(vals)
     out = {

@@ -81,6 +81,14 @@ typedef struct muon_config {
     int param_dtype;                  /* MUON_DTYPE_F32 (default) or MUON_DTYPE_BF16            */
     int grad_dtype;                   /* gradients of muon_step and muon_adamw_step:
                                          MUON_DTYPE_BF16 (default) or MUON_DTYPE_F32            */
+    float soft_threshold;             /* muon_step only: lam of the soft-threshold split (ROOT
+                                         page, "ROOT优化器的技术创新": min ||M - B - O||_F^2 +
+                                         lam ||O||_1, only the robust part B is orthogonalised).
+                                         The outliers O are the update soft-thresholded at
+                                         lam / 2, so B is the update clipped elementwise to
+                                         [-lam/2, lam/2]; the momentum buffer keeps the full
+                                         momentum.  A non-finite update (+-Inf, NaN) still flags
+                                         the matrix non-finite.  0 = off (default); finite, >= 0 */
 } muon_config;
 
 /* Library version (MUON_VERSION of the build). */

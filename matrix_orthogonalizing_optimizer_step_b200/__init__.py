@@ -149,7 +149,7 @@ def _cfg_to_dict(cfg):
         "coeffs": [tuple(cfg.coeffs[3 * k:3 * k + 3]) for k in range(cfg.steps)],
         "mode": cfg.mode, "restart_mask": cfg.restart_mask, "eps": cfg.eps,
         "momentum_dtype": cfg.momentum_dtype, "param_dtype": cfg.param_dtype,
-        "grad_dtype": cfg.grad_dtype,
+        "grad_dtype": cfg.grad_dtype, "soft_threshold": cfg.soft_threshold,
     }
 
 
@@ -160,7 +160,8 @@ def muon_get_config():
 
 
 def muon_set_config(steps=None, coeffs=None, mode=None, restart_mask=None,
-                    eps=None, momentum_dtype=None, param_dtype=None, grad_dtype=None):
+                    eps=None, momentum_dtype=None, param_dtype=None, grad_dtype=None,
+                    soft_threshold=None):
     """Install a config; unspecified fields keep their current values."""
     cfg = _lib.MuonConfig()
     _check(lib().muon_get_config(ctypes.byref(cfg)))
@@ -182,6 +183,8 @@ def muon_set_config(steps=None, coeffs=None, mode=None, restart_mask=None,
         cfg.param_dtype = param_dtype
     if grad_dtype is not None:
         cfg.grad_dtype = grad_dtype
+    if soft_threshold is not None:
+        cfg.soft_threshold = float(soft_threshold)
     _check(lib().muon_set_config(ctypes.byref(cfg)))
 
 

@@ -52,6 +52,7 @@ class MuonConfig(ctypes.Structure):
         ("momentum_dtype", ctypes.c_int),
         ("param_dtype", ctypes.c_int),
         ("grad_dtype", ctypes.c_int),
+        ("soft_threshold", ctypes.c_float),
     ]
 
 

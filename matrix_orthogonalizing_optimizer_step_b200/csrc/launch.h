@@ -66,6 +66,7 @@ struct MomLaunch {
     int nesterov;
     float mu;
     float lr;           // learning rate of a Muon step (0 for orthogonalize)
+    float clip;         // > 0: the update is clipped to [-clip, clip] (soft-threshold split)
     double eps;
     float* partials;    // one per chunk
     int* counters;      // one per matrix, zero between launches

@@ -80,7 +80,7 @@ __device__ __forceinline__ T block_sum(T v, T* red) {
     return r;  // valid in thread 0
 }
 
-template <bool G_F32, int MOM, bool U_F32>
+template <bool G_F32, int MOM, bool U_F32, bool CLIP>
 __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch L) {
     __shared__ float red_f[kThreads / 32];
     __shared__ double red_d[kThreads / 32];
@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     const long long numel = Mx.rows * Mx.cols;
     const long long e0 = (chunk - Mx.chunk_begin) * kMomChunk;
     const float mu = L.mu;
+    const float clip = L.clip;
     float ss = 0.f;
 
     auto step = [&](float g, float& m_io) -> float {
@@ -100,6 +101,15 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
         const float mn = fmaf(mu, m_io, g);
         m_io = mn;
         return L.nesterov ? fmaf(mu, mn, g) : mn;
+    };
+    // Soft-threshold split (CLIP): the update is clipped to [-clip, clip] (the
+    // outlier part is dropped) and the sum of squares is taken of the clipped
+    // values.  u - u is 0 for finite u and NaN for +-Inf or NaN, so a
+    // non-finite update still flags the matrix.
+    auto split = [&](float u, float& acc) -> float {
+        if (!CLIP) return u;
+        acc += __fsub_rn(u, u);
+        return fminf(fmaxf(u, -clip), clip);
     };
 
     if (Mx.vec_ok) {
@@ -112,7 +122,7 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
                 if (MOM != MOM_NONE) load8(Mx.m, MOM == MOM_F32, e, m);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    u[j] = step(g[j], m[j]);
+                    u[j] = split(step(g[j], m[j]), ss);
                     ss = fmaf(u[j], u[j], ss);
                 }
                 if (MOM != MOM_NONE) store8(Mx.m, MOM == MOM_F32, e, m);
@@ -127,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
             const float g = ld_elem(Mx.g, G_F32 ? DT_F32 : DT_BF16, e);
             float m = 0.f;
             if (MOM != MOM_NONE) m = ld_elem(Mx.m, MOM == MOM_F32 ? DT_F32 : DT_BF16, e);
-            const float u = step(g, m);
+            const float u = split(step(g, m), ss);
             ss = fmaf(u, u, ss);
             if (MOM != MOM_NONE) st_elem(Mx.m, MOM == MOM_F32 ? DT_F32 : DT_BF16, e, m);
             st_elem(Mx.u, U_F32 ? DT_F32 : DT_BF16, r * Mx.ldu + c, u);
@@ -195,32 +205,38 @@ __global__ void __launch_bounds__(kThreads) scale_apply_kernel(const ScaleLaunch
 
 }  // namespace
 
+template <bool CLIP>
+static cudaError_t launch_step(const MomLaunch& L, dim3 grid, bool gf, cudaStream_t stream) {
+    if (gf) {
+        if (L.mom_dt == DT_F32)
+            momentum_norm_kernel<true, MOM_F32, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+        else
+            momentum_norm_kernel<true, MOM_BF16, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+    } else {
+        if (L.mom_dt == DT_F32)
+            momentum_norm_kernel<false, MOM_F32, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+        else
+            momentum_norm_kernel<false, MOM_BF16, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream) {
     if (L.nchunks <= 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(L.nchunks));
     const bool gf = L.in_dt == DT_F32, uf = L.u_dt == DT_F32;
     if (!L.has_momentum) {
         if (gf && uf)
-            momentum_norm_kernel<true, MOM_NONE, true><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<true, MOM_NONE, true, false><<<grid, kThreads, 0, stream>>>(L);
         else if (!gf && !uf)
-            momentum_norm_kernel<false, MOM_NONE, false><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<false, MOM_NONE, false, false><<<grid, kThreads, 0, stream>>>(L);
         else
             return cudaErrorInvalidValue;
-    } else {
-        if (uf) return cudaErrorInvalidValue;
-        if (gf) {
-            if (L.mom_dt == DT_F32)
-                momentum_norm_kernel<true, MOM_F32, false><<<grid, kThreads, 0, stream>>>(L);
-            else
-                momentum_norm_kernel<true, MOM_BF16, false><<<grid, kThreads, 0, stream>>>(L);
-        } else {
-            if (L.mom_dt == DT_F32)
-                momentum_norm_kernel<false, MOM_F32, false><<<grid, kThreads, 0, stream>>>(L);
-            else
-                momentum_norm_kernel<false, MOM_BF16, false><<<grid, kThreads, 0, stream>>>(L);
-        }
+        return cudaGetLastError();
     }
-    return cudaGetLastError();
+    if (uf) return cudaErrorInvalidValue;
+    if (L.clip > 0.f) return launch_step<true>(L, grid, gf, stream);
+    return launch_step<false>(L, grid, gf, stream);
 }
 
 cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream) {

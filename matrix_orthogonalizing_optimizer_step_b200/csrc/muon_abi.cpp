@@ -61,6 +61,7 @@ void fill_defaults(muon_config* c) {
     c->momentum_dtype = MUON_DTYPE_BF16;
     c->param_dtype = MUON_DTYPE_F32;
     c->grad_dtype = MUON_DTYPE_BF16;
+    c->soft_threshold = 0.f;
 }
 
 void ensure_cfg() {
@@ -82,6 +83,8 @@ int check_cfg(const muon_config& c) {
         return fail(MUON_ERR_UNSUPPORTED, "config.param_dtype must be BF16 or F32");
     if (c.grad_dtype != MUON_DTYPE_BF16 && c.grad_dtype != MUON_DTYPE_F32)
         return fail(MUON_ERR_UNSUPPORTED, "config.grad_dtype must be BF16 or F32");
+    if (!std::isfinite(c.soft_threshold) || c.soft_threshold < 0.f)
+        return fail(MUON_ERR_INVALID_ARG, "config.soft_threshold must be finite and >= 0");
     return MUON_OK;
 }
 
@@ -197,7 +200,7 @@ int run_plan(DeviceState* ds, const PlanRequest& rq) {
             return fail(st, err);
         }
     }
-    plan.set_scalars(rq.mu, rq.nesterov, rq.lr);
+    plan.set_scalars(rq.mu, rq.nesterov, rq.lr, rq.clip);
     long long launched = 0;
     const int st = plan.run(g_stream, g_prof.on ? &g_prof : nullptr, &launched, err);
     g_launches += launched;
@@ -353,6 +356,7 @@ int muon_step(void* const* params, const void* const* grads, void* const* moment
     rq.mu = mu;
     rq.nesterov = nesterov ? 1 : 0;
     rq.lr = lr;
+    rq.clip = 0.5f * g_cfg.soft_threshold;
     rq.device = ds->device;
     return run_plan(ds, rq);
 }

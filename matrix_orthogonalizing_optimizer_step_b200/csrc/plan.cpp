@@ -344,12 +344,13 @@ static std::vector<long long> make_key(const PlanRequest& rq) {
 
 bool Plan::same_shape_key(const PlanRequest& rq) const { return !key_.empty() && make_key(rq) == key_; }
 
-void Plan::set_scalars(float mu, int nesterov, float lr) {
+void Plan::set_scalars(float mu, int nesterov, float lr, float clip) {
     for (LaunchRec& l : launches) {
         if (l.kind == LaunchRec::MOM) {
             l.mom.mu = mu;
             l.mom.nesterov = nesterov;
             l.mom.lr = lr;
+            l.mom.clip = clip;
         } else if (l.kind == LaunchRec::SCALE) {
             l.sc.lr = lr;
         }
@@ -572,6 +573,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         L.nesterov = rq.nesterov;
         L.mu = rq.mu;
         L.lr = rq.lr;
+        L.clip = rq.clip;
         L.eps = rq.eps;
         L.partials = d_partials;
         L.counters = d_counters;

@@ -35,6 +35,7 @@ struct PlanRequest {
     float mu = 0.95f;
     int nesterov = 1;
     float lr = 0.f;
+    float clip = 0.f;              // muon_step: the update is clipped to [-clip, clip] (0 = off)
     int device = 0;
 };
 
@@ -62,7 +63,7 @@ class Plan {
     // True when `req` differs from the built plan only in mu, nesterov, lr.
     bool same_shape_key(const PlanRequest& req) const;
     // Patch the per-call scalars (mu, nesterov, lr) into the launch records.
-    void set_scalars(float mu, int nesterov, float lr);
+    void set_scalars(float mu, int nesterov, float lr, float clip);
     int run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter, std::string& err);
     void release();
     ~Plan() { release(); }

@@ -47,6 +47,7 @@ def test_version_and_defaults(lib):
     assert cfg["momentum_dtype"] == mo.MUON_DTYPE_BF16
     assert cfg["param_dtype"] == mo.MUON_DTYPE_F32
     assert cfg["grad_dtype"] == mo.MUON_DTYPE_BF16
+    assert cfg["soft_threshold"] == 0.0
 
 
 def test_config_roundtrip_and_validation(lib):
@@ -57,7 +58,8 @@ def test_config_roundtrip_and_validation(lib):
     assert c["steps"] == 3 and c["mode"] == mo.MUON_NS_GRAM and c["restart_mask"] == 2
     assert c["coeffs"][1] == pytest.approx((3, -4, 2))
     for bad in [dict(steps=17), dict(steps=-1), dict(mode=7), dict(eps=float("nan")),
-                dict(momentum_dtype=5), dict(param_dtype=9), dict(grad_dtype=3)]:
+                dict(momentum_dtype=5), dict(param_dtype=9), dict(grad_dtype=3),
+                dict(soft_threshold=-1.0), dict(soft_threshold=float("inf"))]:
         with pytest.raises(mo.MuonError) as e:
             mo.muon_set_config(**bad)
         assert e.value.code in (mo.MUON_ERR_INVALID_ARG, mo.MUON_ERR_UNSUPPORTED)

@@ -105,6 +105,34 @@ def test_step_fp32_gradients(mom_dt):
     _run_and_check(SHAPES[:4] + [(37, 91)], mom_dt=mom_dt, grad_dt="f32")
 
 
+@pytest.mark.parametrize("form", ["standard", "gram"])
+def test_step_soft_threshold_split(form):
+    """ROOT's soft-threshold split: the update is clipped to [-lam/2, lam/2]
+    before orthogonalisation; the momentum buffer keeps the outliers."""
+    lam = 0.06
+    shapes = [(256, 768), (136, 520), (520, 136), (200, 200)]
+    mo.muon_set_config(mode=form, soft_threshold=lam)
+    G = [wl.make_single(r, c, 900 + i, "student_t3_outl", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, 950 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, 990 + i, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    W64, G64, M64 = [to64(t) for t in W], [to64(t) for t in G], [to64(t) for t in M]
+    lr = 0.1
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=lr)
+    torch.cuda.synchronize()
+    for i, (r, c) in enumerate(shapes):
+        W1, M1, O = orc.muon_step(W64[i], G64[i], M64[i], 0.95, True, lr, form=form, soft_threshold=lam)
+        _, _, O_plain = orc.muon_step(W64[i], G64[i], M64[i], 0.95, True, lr, form=form)
+        O_gpu = (W64[i] - to64(W[i])) / lr
+        assert relF(O_gpu, O) <= TOL_BF16_RELF, (shapes[i], relF(O_gpu, O))
+        assert sigma_maxdiff(O_gpu, O) <= TOL_SIGMA
+        # the split changes the update (the outliers are real) ...
+        assert relF(O_plain, O) > 5 * TOL_BF16_RELF
+        # ... and the momentum buffer is the full, unclipped momentum
+        got_m = to64(M[i])
+        assert np.mean(got_m == _expected_momentum(M64[i], G64[i], 0.95, "bf16")) >= 0.9999
+        assert np.max(np.abs(got_m)) > lam  # outliers kept in the buffer
+
+
 def test_step_unaligned_columns():
     _run_and_check([(37, 91), (91, 37), (13, 200)], form="auto")
 
@@ -117,9 +145,14 @@ def test_step_zero_lr_leaves_params():
     assert torch.equal(W[0], W0)
 
 
-def test_step_nonfinite_gradient_leaves_param():
+@pytest.mark.parametrize("bad_value,soft_threshold", [(float("nan"), 0.0), (float("inf"), 0.0),
+                                                     (float("nan"), 0.06), (float("inf"), 0.06)])
+def test_step_nonfinite_gradient_leaves_param(bad_value, soft_threshold):
+    """A non-finite gradient entry flags its matrix and leaves its parameter
+    untouched, also when the soft-threshold split would clip it."""
+    mo.muon_set_config(soft_threshold=soft_threshold)
     W, G, M = _make_set([(64, 192), (96, 96)], 88)
-    G[1][5, 7] = float("nan")
+    G[1][5, 7] = bad_value
     W1 = W[1].clone()
     mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.1)
     st, bad = mo.muon_device_status()

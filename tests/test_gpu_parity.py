@@ -67,7 +67,7 @@ def test_bf16_256x1024(form):
 
 # ---- ragged / edge shapes (several tiles and a ragged tail) ------------------
 
-RAGGED = [(200, 712), (712, 200), (72, 1000), (130, 130), (37, 91), (91, 37), (8, 8), (1, 40),
+RAGGED = [(200, 712), (712, 200), (72, 1000), (130, 130), (37, 91), (91, 37), (8, 8), (1, 40), (1, 1), (2, 3), (3, 2), (1, 4097),
           (40, 1), (384, 1536), (1000, 136), (264, 520), (520, 264), (300, 300)]
 
 

@@ -338,6 +338,15 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         // prefetch the C1 row segment of the first slice while the MMAs run
         Raw32 pre[2];
         prefetch_row32(ep, PM, PN, row, cbase, pre[0]);
+        // C2 (the parameters of the fused update, read once from DRAM): pull
+        // this lane's row of the warp's 128 columns into L2 now, so the
+        // per-slice loads below hit L2
+        if (ep.c2 && !skip && row < PM) {
+            const int es = ep.c2_dt == DT_F32 ? 4 : 2;
+            const char* p = static_cast<const char*>(ep.c2) + (row * ep.ldc2 + cbase) * es;
+            const int bytes = min(BN / 2, PN - cbase) * es;
+            for (int o = 0; o < bytes; o += 128) prefetch_l2(p + o);
+        }
         if (!mbar_wait(&sh->tfull[acc], acc_phase, abort_flag)) {
             if (lane == 0) record_timeout(sh, L.status);
             break;

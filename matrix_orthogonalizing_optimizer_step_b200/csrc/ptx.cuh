@@ -167,6 +167,11 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sm
                  : "memory");
 }
 
+// Pull the 128-byte line holding `p` into L2 (no register result).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // At most N of this thread's bulk groups still read their shared-memory source.

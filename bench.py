@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-adamw", action="store_true",
+                    help="skip the AdamW-lane measurement on the model's AdamW parameters")
     ap.add_argument("--soft-threshold", type=float, default=0.0,
                     help="lam of the soft-threshold split of the update (0 = plain Muon)")
     ap.add_argument("--subset", type=int, default=0,
@@ -254,6 +256,46 @@ def traffic_from_profiles():
         return None
 
 
+def time_adamw_lane(w, dev, steps, peaks, world):
+    """Device time of muon_adamw_step over the model's AdamW parameters (fp32
+    params and moments, bf16 grads: 26 bytes per element), after 3 warm-up
+    steps; GB/s against the measured HBM copy bandwidth."""
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+    numels = list(w.adamw_numels)
+    mo.muon_set_config(param_dtype=mo.MUON_DTYPE_F32, grad_dtype=mo.MUON_DTYPE_BF16)
+    P, G, M1, M2 = [], [], [], []
+    for i, n in enumerate(numels):
+        P.append(wl.make_single(1, n, 5000 + i, "params", dev, "f32").view(-1))
+        G.append(wl.make_single(1, n, 6000 + i, "student_t3", dev, "bf16", 0.01).view(-1))
+        M1.append(torch.zeros(n, device=dev))
+        M2.append(torch.zeros(n, device=dev))
+    t = 0
+    for _ in range(3):
+        t += 1
+        mo.muon_adamw_step(P, G, M1, M2, t)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        t += 1
+        mo.muon_adamw_step(P, G, M1, M2, t)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    elems = sum(numels)
+    gbs = 26.0 * elems / (ms * 1e-3) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    mo.muon_reset_config()
+    del P, G, M1, M2
+    torch.cuda.empty_cache()
+    return {"kernel": "adamw (fused decoupled-decay AdamW, one grouped launch)", "tensors": len(numels),
+            "elements": elems, "ms": round(ms, 4), "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(gbs / peak, 4) if peak else None, "bytes_per_element": 26}
+
+
 def run_ours(args):
     import torch
     import matrix_orthogonalizing_optimizer_step_b200 as mo
@@ -411,6 +453,11 @@ def run_ours(args):
                "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
                "note": "pinned host grads -> HBM, muon_step, params -> pinned host, per step"}
 
+    # ---- the hybrid optimizer's AdamW lane on the model's AdamW parameters ----
+    adamw = None
+    if w.adamw_numels and not args.no_adamw:
+        adamw = time_adamw_lane(w, dev, max(args.steps, 5), peaks, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_step_ms(w, args.cpu_seconds, args.form, args.soft_threshold)
@@ -434,6 +481,7 @@ def run_ours(args):
             "roofline": roofline, "roofline_momentum": roofline_mom,
             "gpu_launches": int(launches),
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
+            "adamw_lane": adamw,
         }
         print(json.dumps(out), flush=True)
     if world > 1:

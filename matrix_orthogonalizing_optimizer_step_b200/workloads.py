@@ -43,6 +43,9 @@ class Workload:
     forms: tuple = ("gram",)
     notes: str = ""
     meta: dict = field(default_factory=dict)
+    # element counts of the model's AdamW parameters (embeddings, output
+    # head, 1-D parameters), empty when the set has no model around it
+    adamw_numels: tuple = ()
 
     @property
     def count(self):
@@ -64,6 +67,20 @@ def _llama8b_shapes():
     return tuple(s for _ in range(32) for s in per_layer)
 
 
+def _gpt2_adamw_numels():
+    # token / position embeddings (the output head is tied to wte), per layer
+    # ln_1 (w, b), qkv bias, attn-out bias, ln_2 (w, b), fc bias, proj bias,
+    # final ln_f (w, b)
+    per_layer = (768, 768, 2304, 768, 768, 768, 3072, 768)
+    return (50257 * 768, 1024 * 768) + per_layer * 12 + (768, 768)
+
+
+def _llama8b_adamw_numels():
+    # token embedding and untied output head (vocabulary 128256), per layer
+    # two RMSNorm gains, final norm
+    return (128256 * 4096, 128256 * 4096) + (4096, 4096) * 32 + (4096,)
+
+
 def _moe_shapes():
     return tuple(s for _ in range(64) for s in ((2048, 7168), (7168, 2048)))
 
@@ -74,7 +91,8 @@ WORKLOADS = {
                 notes="fp32 N(0,1), seed 0; also the fp32 check path"),
     2: Workload(2, "gpt2-124m-muon-set", _gpt2_shapes(), "student_t3", 0.01,
                 notes="12 layers x {qkv 768x2304, attn-out 768x768, "
-                      "fc 768x3072, proj 3072x768}; momentum 0.95 Nesterov"),
+                      "fc 768x3072, proj 3072x768}; momentum 0.95 Nesterov",
+                adamw_numels=_gpt2_adamw_numels()),
     3: Workload(3, "aspect-sweep-b16",
                 tuple([(2048, 2048)] * 16 + [(2048, 8192)] * 16
                       + [(1024, 16384)] * 16),
@@ -84,7 +102,8 @@ WORKLOADS = {
                       "Gram NS with restart"),
     5: Workload(5, "llama-8b-muon-set", _llama8b_shapes(), "normal_1e-4",
                 notes="32 layers x {q,o 4096x4096; k,v 4096x1024; "
-                      "gate,up 4096x14336; down 14336x4096}"),
+                      "gate,up 4096x14336; down 14336x4096}",
+                adamw_numels=_llama8b_adamw_numels()),
 }
 
 _TORCH_DTYPE = {"bf16": torch.bfloat16, "f32": torch.float32,

@@ -6,7 +6,7 @@
 //     m <- b1 m + (1 - b1) g ;  v <- b2 v + (1 - b2) g^2
 //     p <- p - lr (m c1) / (sqrt(v c2) + eps),  c1 = 1/(1 - b1^t), c2 = 1/(1 - b2^t)
 // One grouped launch over all tensors: one CTA per chunk of 8192 elements of
-// one tensor, 4-element vector access when aligned.  HBM-bound: 26 bytes per
+// one tensor, 8-element vector access when aligned.  HBM-bound: 26 bytes per
 // element with fp32 parameters and bf16 gradients (p, m, v read and written, g read).
 #include <cuda_bf16.h>
 
@@ -53,45 +53,40 @@ __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
     const AdamCoef k{L.decay, L.beta1, 1.f - L.beta1, L.beta2, 1.f - L.beta2, L.lr_c1, L.c2, L.eps};
     const int pdt = P_F32 ? DT_F32 : DT_BF16;
     if (T.vec_ok) {
-        for (int i = threadIdx.x; i < kMomChunk / 4; i += kThreads) {
-            const long long e = e0 + 4LL * i;
+        // 8 elements per thread and iteration: two 16-byte accesses per fp32
+        // array, one per 16-bit array
+        for (int i = threadIdx.x; i < kMomChunk / 8; i += kThreads) {
+            const long long e = e0 + 8LL * i;
             if (e >= T.numel) break;
-            float p[4], g[4];
-            if (P_F32) {
-                const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(T.p) + e);
-                p[0] = q.x, p[1] = q.y, p[2] = q.z, p[3] = q.w;
-            } else {
-                const uint2 q = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(T.p) + e);
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-                p[0] = a.x, p[1] = a.y, p[2] = b.x, p[3] = b.y;
-            }
-            if (G_F32) {
-                const float4 q = *reinterpret_cast<const float4*>(static_cast<const float*>(T.g) + e);
-                g[0] = q.x, g[1] = q.y, g[2] = q.z, g[3] = q.w;
-            } else {
-                const uint2 q = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(T.g) + e);
-                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.x));
-                const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q.y));
-                g[0] = a.x, g[1] = a.y, g[2] = b.x, g[3] = b.y;
-            }
-            float4 m = *reinterpret_cast<const float4*>(T.m + e);
-            float4 v = *reinterpret_cast<const float4*>(T.v + e);
-            p[0] = adam_elem(p[0], g[0], m.x, v.x, k);
-            p[1] = adam_elem(p[1], g[1], m.y, v.y, k);
-            p[2] = adam_elem(p[2], g[2], m.z, v.z, k);
-            p[3] = adam_elem(p[3], g[3], m.w, v.w, k);
-            *reinterpret_cast<float4*>(T.m + e) = m;
-            *reinterpret_cast<float4*>(T.v + e) = v;
-            if (P_F32) {
-                *reinterpret_cast<float4*>(static_cast<float*>(T.p) + e) = make_float4(p[0], p[1], p[2], p[3]);
-            } else {
-                __nv_bfloat162 a = __floats2bfloat162_rn(p[0], p[1]), b = __floats2bfloat162_rn(p[2], p[3]);
-                uint2 q;
-                q.x = *reinterpret_cast<uint32_t*>(&a);
-                q.y = *reinterpret_cast<uint32_t*>(&b);
-                *reinterpret_cast<uint2*>(static_cast<uint16_t*>(T.p) + e) = q;
-            }
+            float p[8], g[8], m[8], v[8];
+            auto ld8f = [](const float* src, float* dst) {
+                const float4 a = *reinterpret_cast<const float4*>(src);
+                const float4 b = *reinterpret_cast<const float4*>(src + 4);
+                dst[0] = a.x, dst[1] = a.y, dst[2] = a.z, dst[3] = a.w;
+                dst[4] = b.x, dst[5] = b.y, dst[6] = b.z, dst[7] = b.w;
+            };
+            auto st8f = [](float* dst, const float* src) {
+                *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(src[4], src[5], src[6], src[7]);
+            };
+            if (P_F32)
+                ld8f(static_cast<const float*>(T.p) + e, p);
+            else
+                unpack8(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(T.p) + e), DT_BF16, p);
+            if (G_F32)
+                ld8f(static_cast<const float*>(T.g) + e, g);
+            else
+                unpack8(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(T.g) + e), DT_BF16, g);
+            ld8f(T.m + e, m);
+            ld8f(T.v + e, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) p[j] = adam_elem(p[j], g[j], m[j], v[j], k);
+            st8f(T.m + e, m);
+            st8f(T.v + e, v);
+            if (P_F32)
+                st8f(static_cast<float*>(T.p) + e, p);
+            else
+                *reinterpret_cast<uint4*>(static_cast<uint16_t*>(T.p) + e) = pack8(p, DT_BF16);
         }
     } else {
         for (int i = threadIdx.x; i < kMomChunk; i += kThreads) {

@@ -99,7 +99,7 @@ struct AdamTensor {
     float* v;         // second moment (fp32)
     long long numel;
     long long chunk_begin;
-    int vec_ok;       // numel % 4 == 0 and every pointer aligned for 4-element access
+    int vec_ok;       // numel % 8 == 0 and every pointer 16-byte aligned (8-element access)
 };
 
 struct AdamLaunch {

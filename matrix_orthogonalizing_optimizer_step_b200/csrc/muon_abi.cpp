@@ -387,8 +387,8 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
         t[i].numel = numels[i];
         t[i].chunk_begin = chunks;
         auto al = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
-        t[i].vec_ok = numels[i] % 4 == 0 && al(params[i], pf32 ? 16 : 8) && al(grads[i], gf32 ? 16 : 8) &&
-                      al(exp_avg[i], 16) && al(exp_avg_sq[i], 16);
+        t[i].vec_ok = numels[i] % 8 == 0 && al(params[i], 16) && al(grads[i], 16) && al(exp_avg[i], 16) &&
+                      al(exp_avg_sq[i], 16);
         chunks += (numels[i] + kMomChunk - 1) / kMomChunk;
     }
     DeviceState* ds = nullptr;

@@ -188,6 +188,35 @@ def test_step_deterministic_and_resumable():
         assert torch.equal(x, y)
 
 
+@pytest.mark.parametrize("env", [{"MUON_SLOT_LAUNCHES": "1"}, {"MUON_TMA_STORE": "0"}])
+def test_launch_modes_are_bitwise_equal(env, monkeypatch):
+    """The chained launch and one launch per chain slot, and the TMA-store and
+    plain-store epilogues, compute the same tiles with the same arithmetic:
+    their results are bitwise equal."""
+    shapes = [(768, 2304), (768, 768), (3072, 768), (200, 712), (37, 91)]
+
+    def run():
+        W, G, M = _make_set(shapes, 1200)
+        for _ in range(2):
+            mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.02)
+        torch.cuda.synchronize()
+        return [t.clone() for t in W + M]
+
+    monkeypatch.setenv("MUON_CHAIN_LAUNCH", "1")
+    mo.muon_release_workspace()  # the launch mode is chosen when a plan is built
+    ref = run()
+    monkeypatch.delenv("MUON_CHAIN_LAUNCH")
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    mo.muon_release_workspace()
+    got = run()
+    for k in env:
+        monkeypatch.delenv(k)
+    mo.muon_release_workspace()
+    for x, y in zip(ref, got):
+        assert torch.equal(x, y)
+
+
 def test_profile_counts_match_oracle_flops():
     shapes = [(256, 768), (768, 256), (512, 512)]
     W, G, M = _make_set(shapes, 500)

@@ -1,7 +1,7 @@
 """fp64 CPU oracle for the Muon step.  Test infrastructure only: never imported
 by the product path (see muon_oracle's header)."""
 from .muon_oracle import (  # noqa: F401
-    BASELINE_COEFFS,
+    CLASSIC_COEFFS,
     DEFAULT_EPS,
     DEFAULT_RESTARTS,
     TUNED_COEFFS,

@@ -24,7 +24,7 @@ Sources (web pages; formulas were lost in extraction, the prose survives):
   FLOP 开销分析" (coefficients (3.4445, -4.7750, 2.0315), five steps, older
   (2, -1.5, 0.5)), "工程复现清单" (momentum 0.95, nesterov=True, lr 6e-4).
 
-Readings where the sources are silent (each listed in the design doc):
+Readings where the sources are silent:
 
 * momentum: M <- mu*M + G; Nesterov U = G + mu*M, else U = M;
 * Frobenius normalisation X0 = U / (||U||_F + eps), eps = 1e-7;
@@ -39,7 +39,7 @@ from __future__ import annotations
 import numpy as np
 
 TUNED_COEFFS = (3.4445, -4.7750, 2.0315)
-BASELINE_COEFFS = (2.0, -1.5, 0.5)
+CLASSIC_COEFFS = (2.0, -1.5, 0.5)
 DEFAULT_EPS = 1e-7
 DEFAULT_RESTARTS = (2,)
 

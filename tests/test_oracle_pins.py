@@ -47,7 +47,7 @@ def _relF(a, b):
 
 
 SHAPES = [(24, 40), (32, 32), (40, 24), (7, 61)]
-COEFFS = [orc.TUNED_COEFFS, orc.BASELINE_COEFFS,
+COEFFS = [orc.TUNED_COEFFS, orc.CLASSIC_COEFFS,
           # per-step coefficients (one triple per step)
           ((3.4445, -4.7750, 2.0315), (2.9, -4.0, 1.9), (2.5, -3.0, 1.4),
            (2.0, -1.5, 0.5), (1.875, -1.25, 0.375))]
@@ -74,7 +74,7 @@ def test_gram_equals_standard(restarts, steps):
     assert _relF(gram, std) < 1e-12
 
 
-def test_baseline_coefficients_converge_to_polar():
+def test_classic_coefficients_converge_to_polar():
     X = _rng(3).standard_normal((48, 80))
     U, S, Vt = np.linalg.svd(X, full_matrices=False)
     # spread the singular values over [1e-3, 1] to exercise the slow end
@@ -82,7 +82,7 @@ def test_baseline_coefficients_converge_to_polar():
     X = (U * S) @ Vt
     polar = U @ Vt
     for form in ("standard", "gram"):
-        got = orc.orthogonalize(X, orc.BASELINE_COEFFS, 40, form,
+        got = orc.orthogonalize(X, orc.CLASSIC_COEFFS, 40, form,
                                 restarts=(10, 20, 30))
         assert np.max(np.abs(got - polar)) < 1e-10
         sv = np.linalg.svd(got, compute_uv=False)

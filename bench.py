@@ -411,6 +411,10 @@ def run_ours(args):
         "share_of_step": round(momk.get("total_ms", 0) / ms_total, 4) if ms_total else None,
     }
     ns_tflops = gemm.get("flops", 0) / (ms_total * 1e-3) / 1e12 if ms_total else 0.0
+    # the standard form's work for the same matrices (15 n^2 m + 5 n^3 each, symmetric
+    # products at half cost) over the same time: comparable across NS forms
+    std_flops = sum(15.0 * min(r, c) ** 2 * max(r, c) + 5.0 * min(r, c) ** 3 for r, c in w.shapes)
+    ns_tflops_std = std_flops * args.steps / (ms_total * 1e-3) / 1e12 if ms_total else 0.0
 
     # ---- end to end through the public API, host buffers ---------------------
     e2e = None
@@ -478,6 +482,7 @@ def run_ours(args):
                        "l2": f"inputs larger than L2: {in_bytes_resident / 1e6:.0f} MB read per step",
                        "parallelism": f"replica x{world} (independent per GPU)"},
             "ns_tflops_per_step": round(ns_tflops, 2),
+            "ns_tflops_standard_equivalent": round(ns_tflops_std, 2),
             "roofline": roofline, "roofline_momentum": roofline_mom,
             "gpu_launches": int(launches),
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,

@@ -336,8 +336,8 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         const int nbox = ep.o1_dt == DT_F32 ? 2 : 1;  // 64-byte boxes per 32-column slice
         bool stored = false;
         // prefetch the C1 row segment of the first slice while the MMAs run
-        Raw32 pre[2];
-        prefetch_row32(ep, PM, PN, row, cbase, pre[0]);
+        Raw32 pre;
+        prefetch_row32(ep, PM, PN, row, cbase, pre);
         // C2 (the parameters of the fused update, read once from DRAM): pull
         // this lane's row of the warp's 128 columns into L2 now, so the
         // per-slice loads below hit L2
@@ -352,22 +352,31 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             break;
         }
         tc_fence_after();
-#pragma unroll
+        // one slice per iteration, not unrolled: the epilogue's code stays small
+#pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
             const int col0 = cbase + c;
-            const int cur = (c / 32) & 1;
-            if (c + 32 < BN / 2) prefetch_row32(ep, PM, PN, row, col0 + 32, pre[cur ^ 1]);
-            if (col0 >= PN) continue;  // warp-uniform
+            Raw32 nxt;  // C1 of the next slice, fetched while this one is processed
+            nxt.ok = 0;
+            if (c + 32 < BN / 2) prefetch_row32(ep, PM, PN, row, col0 + 32, nxt);
+            if (col0 >= PN) {  // warp-uniform
+                pre = nxt;
+                continue;
+            }
             uint32_t r[32];
             __syncwarp();
             tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * (BN / 2) + c,
                                r);
             tmem_wait_ld();
-            if (skip || row0 >= PM) continue;  // warp-uniform
+            if (skip || row0 >= PM) {  // warp-uniform
+                pre = nxt;
+                continue;
+            }
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-            const bool valid = epilogue_values32(ep, sig, PM, PN, row, col0, v, &pre[cur]);
+            const bool valid = epilogue_values32(ep, sig, PM, PN, row, col0, v, &pre);
+            pre = nxt;
             if (!use_tma) {
                 if (valid) store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, 0, min(32, PN - col0), v);
                 continue;

@@ -58,6 +58,20 @@ __device__ __forceinline__ uint4 pack8(const float* v, int dt) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 32 values passed by value to the out-of-line (cold) element-wise paths, so
+// that the hot paths' register arrays never need an address.
+struct Row32 {
+    float v[32];
+};
+
+// Element-wise load of a ragged or unaligned row segment (cold path).
+static __device__ __noinline__ Row32 load_row32_elems(const void* base, int dt, long long off, int nvalid) {
+    Row32 r;
+#pragma unroll 4
+    for (int j = 0; j < 32; ++j) r.v[j] = (j < nvalid) ? ld_elem(base, dt, off + j) : 0.f;
+    return r;
+}
+
 // Load 32 consecutive elements of one row (columns col0 .. col0+31); columns
 // at or beyond col0 + nvalid read as 0.
 __device__ __forceinline__ void load_row32(const void* base, int dt, long long ld, long long row, int col0,
@@ -81,8 +95,9 @@ __device__ __forceinline__ void load_row32(const void* base, int dt, long long l
         }
         return;
     }
+    const Row32 r = load_row32_elems(base, dt, off, nvalid);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) out[j] = (j < nvalid) ? ld_elem(base, dt, off + j) : 0.f;
+    for (int j = 0; j < 32; ++j) out[j] = r.v[j];
 }
 
 // Store columns [jmin, nvalid) of a 32-wide row segment (one lane's row).
@@ -106,6 +121,13 @@ __device__ __forceinline__ void store_row32(void* base, int dt, long long ld, lo
 #pragma unroll
     for (int j = 0; j < 32; ++j)
         if (j >= jmin && j < nvalid) st_elem(base, dt, off + j, v[j]);
+}
+
+// store_row32 for outputs that TMA cannot store (unaligned row pitch): a cold
+// path, kept out of line.
+static __device__ __noinline__ void store_row32_cold(void* base, int dt, long long ld, long long row, int col0, int nvalid,
+                                              Row32 v) {
+    store_row32(base, dt, ld, row, col0, 0, nvalid, v.v);
 }
 
 // C1 row segment fetched ahead of its use (16-bit C1, aligned, fully in range).

@@ -378,7 +378,12 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             const bool valid = epilogue_values32(ep, sig, PM, PN, row, col0, v, &pre);
             pre = nxt;
             if (!use_tma) {
-                if (valid) store_row32(ep.o1, ep.o1_dt, ep.ldo1, row, col0, 0, min(32, PN - col0), v);
+                if (valid) {
+                    Row32 out;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) out.v[j] = v[j];
+                    store_row32_cold(ep.o1, ep.o1_dt, ep.ldo1, row, col0, min(32, PN - col0), out);
+                }
                 continue;
             }
             // staged TMA store: rows past M and columns past N are clipped

@@ -129,8 +129,9 @@ MUON_API int muon_device_status(int* bad_index);
  * m, n    rows and columns of each matrix (>= 1); the iteration uses the
  *         shorter side (Gram matrix min(m,n) x min(m,n))
  * X       device pointer, in place; bf16 by default, fp32 with MUON_PREC_FP32.
- *         bf16 X must be 16-byte aligned when n % 8 == 0 (any alignment
- *         otherwise: a padded internal copy is used)
+ *         Any alignment: a 16-byte aligned X with n % 8 == 0 takes the
+ *         vectorised loads and the TMA stores, any other X element-wise
+ *         loads and plain stores
  * coeffs  host array of 3*steps floats, (a, b, c) of step k at [3k..3k+2]
  * steps   T in 0..MUON_MAX_STEPS; 0 returns the normalised X
  * mode    MUON_NS_STANDARD | MUON_NS_GRAM | MUON_NS_AUTO, optionally | MUON_PREC_FP32
@@ -148,10 +149,12 @@ MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* c
  * grads       host array of count device pointers, grad_dtype (bf16 default), read only
  * momentum    host array of count device pointers, momentum_dtype, updated in place
  * shape_list  host int[2*count]: rows_i, cols_i of parameter i (>= 1)
- * Coefficients, steps, NS form, restarts, eps and dtypes come from the
- * installed config.  Pointers must be 16-byte aligned for the vectorised
- * path (otherwise a scalar path is used).  Distinct parameters must not
- * overlap.
+ * With muon_config.soft_threshold = lam > 0, U is first clipped elementwise
+ * to [-lam/2, lam/2] (its soft-thresholded outlier part is dropped; M keeps
+ * it).  Coefficients, steps, NS form, restarts, eps, dtypes and the
+ * threshold come from the installed config.  16-byte aligned pointers and
+ * cols % 8 == 0 take the vectorised paths (otherwise element-wise ones).
+ * Distinct parameters must not overlap.
  */
 MUON_API int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
               float lr, const int* shape_list, int count);
@@ -171,8 +174,8 @@ MUON_API int muon_step(void* const* params, const void* const* grads, void* cons
  * numels      host array of count element counts (>= 1); tensors are treated as flat
  * step        the step being taken (>= 1) for the bias corrections
  * 0 <= beta1, beta2 < 1; lr, weight_decay, eps finite (eps >= 0).  One grouped
- * launch on the bound stream; 4-element vector access when every pointer of a
- * tensor is aligned and its numel is a multiple of 4.
+ * launch on the bound stream; 8-element vector access when every pointer of a
+ * tensor is 16-byte aligned and its numel is a multiple of 8.
  */
 MUON_API int muon_adamw_step(void* const* params, const void* const* grads, void* const* exp_avg,
                              void* const* exp_avg_sq, const long long* numels, int count, float lr, float beta1,

@@ -81,6 +81,25 @@ def test_ragged_bf16(shape, form):
     _check(to64(Y), ref, TOL_BF16_RELF)
 
 
+@pytest.mark.parametrize("shape", [(256, 768), (768, 256)])
+@pytest.mark.parametrize("form", ["standard", "gram"])
+def test_misaligned_base_bf16(shape, form):
+    """X starting one element past a 16-byte boundary (width a multiple of 8):
+    element-wise loads and plain stores, same result; nothing outside X is
+    written."""
+    r, c = shape
+    X0 = wl.make_single(r, c, 4242 + r, "gaussian", DEV, "bf16")
+    buf = torch.full((r * c + 16,), 7.0, dtype=torch.bfloat16, device=DEV)
+    X = buf[1:1 + r * c].view(r, c)
+    assert X.data_ptr() % 16 != 0
+    X.copy_(X0)
+    ref = orc.orthogonalize(to64(X0), orc.TUNED_COEFFS, 5, form)
+    mo.muon_orthogonalize(X, steps=5, mode=form)
+    torch.cuda.synchronize()
+    _check(to64(X), ref, TOL_BF16_RELF)
+    assert float(buf[0]) == 7.0 and bool((buf[1 + r * c:] == 7.0).all())
+
+
 @pytest.mark.parametrize("shape", [(200, 712), (712, 200), (37, 91), (300, 300)])
 @pytest.mark.parametrize("form", ["standard", "gram"])
 def test_ragged_fp32(shape, form):

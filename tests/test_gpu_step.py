@@ -137,6 +137,38 @@ def test_step_unaligned_columns():
     _run_and_check([(37, 91), (91, 37), (13, 200)], form="auto")
 
 
+def test_step_misaligned_base_pointers():
+    """Parameters, gradients and momentum starting one element past a 16-byte
+    boundary (widths a multiple of 8) take the element-wise and plain-store
+    paths and give the same step."""
+    shapes = [(256, 768), (768, 256)]
+    W, G, M = [], [], []
+    W64, G64, M64 = [], [], []
+    for i, (r, c) in enumerate(shapes):
+        g0 = wl.make_single(r, c, 3000 + i, "student_t3", DEV, "bf16", 0.01)
+        m0 = wl.make_single(r, c, 3100 + i, "student_t3", DEV, "bf16", 0.01)
+        w0 = wl.make_single(r, c, 3200 + i, "params", DEV, "f32")
+        views = []
+        for t0 in (w0, g0, m0):
+            buf = torch.zeros(r * c + 8, dtype=t0.dtype, device=DEV)
+            v = buf[1:1 + r * c].view(r, c)
+            v.copy_(t0)
+            assert v.data_ptr() % 16 != 0
+            views.append(v)
+        W.append(views[0]), G.append(views[1]), M.append(views[2])
+        W64.append(to64(w0)), G64.append(to64(g0)), M64.append(to64(m0))
+    lr = 0.1
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=lr)
+    torch.cuda.synchronize()
+    for i, (r, c) in enumerate(shapes):
+        n, m = min(r, c), max(r, c)
+        fm = "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
+        _, M1, O = orc.muon_step(W64[i], G64[i], M64[i], 0.95, True, lr, form=fm)
+        O_gpu = (W64[i] - to64(W[i])) / lr
+        assert relF(O_gpu, O) <= TOL_BF16_RELF, (shapes[i], relF(O_gpu, O))
+        assert np.mean(to64(M[i]) == _expected_momentum(M64[i], G64[i], 0.95, "bf16")) >= 0.9999
+
+
 def test_step_zero_lr_leaves_params():
     W, G, M = _make_set([(96, 160)], 77)
     W0 = W[0].clone()

@@ -93,7 +93,7 @@ def ns_standard(X, coeffs=TUNED_COEFFS, steps=5):
     return X
 
 
-def ns_gram(X, coeffs=TUNED_COEFFS, steps=5, restarts=DEFAULT_RESTARTS):
+def ns_gram(X, coeffs=TUNED_COEFFS, steps=5, restarts=DEFAULT_RESTARTS, return_q=False):
     """Gram Newton-Schulz with restarts on X (n x m, n <= m).
 
     [Gram-NS] "ข้อได้เปรียบของอัลกอริทึม": the odd polynomial is p(t) = t q(t^2),
@@ -105,7 +105,8 @@ def ns_gram(X, coeffs=TUNED_COEFFS, steps=5, restarts=DEFAULT_RESTARTS):
     [Gram-NS] "ความท้าทายด้านความเสถียรและแนวทางแก้ไข": a restart re-forms the
     Gram matrix from the current iterate: X <- Q X, R <- X X^T, Q <- I.
     ``restarts`` lists the step indices k (0 < k < steps) at which that
-    happens before step k is taken.  The output is Q X.
+    happens before step k is taken.  The output is Q X (with return_q, also
+    the last segment's Q and the X it multiplies).
     """
     X = np.asarray(X, dtype=np.float64).copy()
     n = X.shape[0]
@@ -120,6 +121,8 @@ def ns_gram(X, coeffs=TUNED_COEFFS, steps=5, restarts=DEFAULT_RESTARTS):
         Z = a * I + b * R + c * (R @ R)
         Q = Z @ Q
         R = Z @ R @ Z
+    if return_q:
+        return Q @ X, Q, X
     return Q @ X
 
 

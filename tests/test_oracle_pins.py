@@ -410,3 +410,29 @@ def test_soft_threshold_muon_step_orthogonalises_the_clipped_update():
     # without the split the outlier dominates: the two updates differ
     _, _, O_plain = orc.muon_step(W, G, M, 0.9, True, 0.1, form="standard")
     assert np.linalg.norm(O - O_plain) > 0.1
+
+
+@pytest.mark.parametrize("shape", [(16, 48), (24, 24), (7, 90)])
+def test_gram_q_closed_form(shape):
+    """[Gram-NS] "ข้อได้เปรียบของอัลกอริทึม": the Gram iteration's Q is a
+    polynomial in R0 = X0 X0^T that approximates R0^{-1/2}.  Without restarts,
+    in R0's eigenbasis (eigenvalues l = sigma^2) Q is diagonal with entries
+    f(sigma) / sigma, f the composed quintic: checked against numpy's
+    symmetric eigendecomposition."""
+    r = _rng(40 + shape[0])
+    X = r.standard_normal(shape)
+    X /= np.linalg.norm(X)
+    _, Q, X_last = orc.ns_gram(X, orc.TUNED_COEFFS, 5, restarts=(), return_q=True)
+    assert np.array_equal(X_last, X)
+    lam, V = np.linalg.eigh(X @ X.T)
+    sigma = np.sqrt(np.maximum(lam, 0.0))
+    f = sigma.copy()
+    for _ in range(5):
+        a, b, c = orc.TUNED_COEFFS
+        f = a * f + b * f ** 3 + c * f ** 5
+    expect = V @ np.diag(f / sigma) @ V.T
+    assert np.allclose(Q, expect, rtol=1e-9, atol=1e-9 * np.abs(expect).max())
+    # with the classic coefficients and many steps, Q -> R0^{-1/2}
+    _, Q40, _ = orc.ns_gram(X, orc.CLASSIC_COEFFS, 40, restarts=(), return_q=True)
+    inv_sqrt = V @ np.diag(1.0 / sigma) @ V.T
+    assert np.allclose(Q40, inv_sqrt, rtol=1e-6, atol=1e-6 * np.abs(inv_sqrt).max())

@@ -122,3 +122,27 @@ def test_profile_api_without_device(lib):
     assert set(stats) == {"momentum_norm", "gemm_tc", "gemm_f32", "scale_apply", "adamw"}
     assert all(v["launches"] == 0 for v in stats.values())
     assert mo.muon_launch_count() >= 0
+
+
+def test_binding_validates_before_calling_the_library():
+    """The Python binding rejects malformed arguments itself (no device is
+    touched): list lengths, dimensions, shapes, contiguity, device, dtype."""
+    import torch
+    a = torch.zeros(4, 8, dtype=torch.bfloat16)
+    b = torch.zeros(4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mo.muon_step([a], [b, b], [a])                       # list lengths differ
+    with pytest.raises(ValueError):
+        mo.muon_step([], [], [])                              # empty
+    with pytest.raises(ValueError):
+        mo.muon_step([torch.zeros(32)], [torch.zeros(32)], [torch.zeros(32)])  # not 2D
+    with pytest.raises(ValueError):
+        mo.muon_step([a], [torch.zeros(8, 4, dtype=torch.bfloat16)], [a])      # shape mismatch
+    with pytest.raises(ValueError):
+        mo.muon_step([a], [torch.zeros(8, 4, dtype=torch.bfloat16).t()], [a])  # not contiguous
+    with pytest.raises(ValueError):
+        mo.muon_orthogonalize(a)                              # not a CUDA tensor
+    with pytest.raises(ValueError):
+        mo.muon_adamw_step([torch.zeros(8)], [torch.zeros(9)], [torch.zeros(8)], [torch.zeros(8)], 1)
+    with pytest.raises(ValueError):
+        mo.muon_adamw_step([torch.zeros(8)], [], [torch.zeros(8)], [torch.zeros(8)], 1)

@@ -7,9 +7,11 @@
 One step = one full Muon step over the workload's 2D parameters (momentum,
 Newton-Schulz, update) through the library's C ABI, or one batched
 orthogonalisation for the NS-only workloads.  Inputs are seeded synthetic
-tensors resident in HBM; the default workload (GPT-2 124M Muon set: 48
-matrices, 85 M elements, ~680 MB of params + grads + momentum per step) is
-larger than the 126 MB L2, so no flush is needed between steps.
+tensors resident in HBM.  The default workload is the largest set, the
+Llama-8B Muon set (224 matrices, 6.98 G elements, ~56 GB of params + grads +
+momentum read per step), far larger than the 126 MB L2, so no flush is
+needed between steps.  A short device-timed measurement of the GPT-2 124M
+set follows as an extra key (--also 0 turns it off).
 
 Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own
 replica of the workload (weak scaling, no data-path collective) and the
@@ -40,7 +42,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--form", default="auto", choices=["auto", "standard", "gram"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -50,6 +52,8 @@ def parse():
                     help="skip the AdamW-lane measurement on the model's AdamW parameters")
     ap.add_argument("--soft-threshold", type=float, default=0.0,
                     help="lam of the soft-threshold split of the update (0 = plain Muon)")
+    ap.add_argument("--also", default="2",
+                    help="comma-separated workload ids timed on the device after the main one (extra key)")
     ap.add_argument("--subset", type=int, default=0,
                     help="use only the first N matrices of the workload (small profiling cases)")
     return ap.parse_args()
@@ -74,52 +78,64 @@ def _ns_form_for(n, m, form):
     return "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
 
 
-def cpu_oracle_step_ms(w, budget_s, form="auto", soft_threshold=0.0):
-    """Time the fp64 oracle on a bounded sample of one step of workload w and
-    scale to the whole step.  Matrices are taken in order (one of each shape
-    first) until the time budget is spent; the per-shape mean time is
-    multiplied by that shape's count."""
-    import numpy as np
-    import torch
-    from oracle import muon_oracle as orc
+def _host_cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # noqa: BLE001
-        cores = os.cpu_count() or 1
-    shapes = list(w.shapes)
-    order, seen = [], set()
-    for i, s in enumerate(shapes):
-        if s not in seen:
-            seen.add(s)
-            order.append(i)
-    order += [i for i in range(len(shapes)) if i not in set(order)]
+        return os.cpu_count() or 1
+
+
+def _distinct_shapes(w):
+    """[(shape, [matrix indices])] in first-appearance order."""
+    by = {}
+    for i, s in enumerate(w.shapes):
+        by.setdefault(s, []).append(i)
+    return list(by.items())
+
+
+def _oracle_seconds(w, i, form, soft_threshold):
+    """Wall seconds of the fp64 oracle on matrix i of workload w (one Muon
+    step of that matrix, or its orthogonalisation for the NS-only sets);
+    input generation is outside the timed part."""
+    import torch
+    from oracle import muon_oracle as orc
+    r, c = w.shapes[i]
+    G = wl.make_matrix(w, i, wl.ROLE_GRAD).to(torch.float64).numpy()
+    fm = _ns_form_for(min(r, c), max(r, c), form)
+    if w.full_step:
+        M = wl.make_matrix(w, i, wl.ROLE_MOMENTUM).to(torch.float64).numpy()
+        W = wl.make_matrix(w, i, wl.ROLE_PARAM).to(torch.float64).numpy()
+        t0 = time.perf_counter()
+        orc.muon_step(W, G, M, 0.95, True, 6e-4, form=fm, soft_threshold=soft_threshold)
+    else:
+        t0 = time.perf_counter()
+        orc.orthogonalize(G, form=fm)
+    return time.perf_counter() - t0
+
+
+def _extrapolate_ms(w, per_shape):
+    return sum(1e3 * statistics.fmean(per_shape[s]) * len(idx) for s, idx in _distinct_shapes(w))
+
+
+def cpu_oracle_step_ms(w, budget_s, form="auto", soft_threshold=0.0):
+    """Time the fp64 oracle on a bounded sample of one step of workload w and
+    scale to the whole step.  One matrix of every distinct shape is timed
+    first, then further matrices in order until the time budget is spent; the
+    per-shape mean time is multiplied by that shape's count."""
+    groups = _distinct_shapes(w)
+    order = [idx[0] for _, idx in groups] + [i for _, idx in groups for i in idx[1:]]
     per_shape = {}
     t_start = time.perf_counter()
     done = 0
     for i in order:
-        if done and time.perf_counter() - t_start > budget_s and all(s in per_shape for s in seen):
+        if done >= len(groups) and time.perf_counter() - t_start > budget_s:
             break
-        r, c = shapes[i]
-        G = wl.make_matrix(w, i, wl.ROLE_GRAD).to(torch.float64).numpy()
-        n, m = min(r, c), max(r, c)
-        fm = _ns_form_for(n, m, form)
-        t0 = time.perf_counter()
-        if w.full_step:
-            M = wl.make_matrix(w, i, wl.ROLE_MOMENTUM).to(torch.float64).numpy()
-            W = wl.make_matrix(w, i, wl.ROLE_PARAM).to(torch.float64).numpy()
-            orc.muon_step(W, G, M, 0.95, True, 6e-4, form=fm, soft_threshold=soft_threshold)
-        else:
-            orc.orthogonalize(G, form=fm)
-        per_shape.setdefault((r, c), []).append(time.perf_counter() - t0)
+        per_shape.setdefault(w.shapes[i], []).append(_oracle_seconds(w, i, form, soft_threshold))
         done += 1
-    total_ms = 0.0
-    for s in seen:
-        cnt = sum(1 for x in shapes if x == s)
-        total_ms += 1e3 * statistics.fmean(per_shape[s]) * cnt
-    sample = (f"{done} of {len(shapes)} matrices (one of each of {len(seen)} shapes first), "
-              f"fp64 NumPy oracle, per-shape mean time x count")
-    return total_ms, cores, sample
+    sample = (f"{done} of {w.count} matrices (one of each of {len(groups)} shapes first), "
+              f"fp64 NumPy oracle, per-shape mean time x count (extrapolated to the whole step)")
+    return _extrapolate_ms(w, per_shape), _host_cores(), sample
 
 
 # ---------------------------------------------------------------------------
@@ -236,10 +252,17 @@ def kernel_sources_hash():
     return h.hexdigest()[:16]
 
 
-def traffic_from_profiles():
-    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel sources (else None)."""
-    p = os.path.join(HERE, "profiles", "gemm_tc_gpt2_traffic.txt")
+def _slug(name):
+    return name.replace("/", "-")
+
+
+def traffic_from_profiles(workload_name):
+    """DRAM bytes per launch of the dominant kernel for this workload, from the
+    committed ncu record profiles/gemm_tc_<workload>_traffic.txt, if that
+    record was taken on the current kernel sources (else None).  A record
+    captured on a subset of the workload states its scaling to the full set
+    and stores the scaled figure (dram_bytes_per_launch)."""
+    p = os.path.join(HERE, "profiles", f"gemm_tc_{_slug(workload_name)}_traffic.txt")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -248,6 +271,8 @@ def traffic_from_profiles():
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
+    if vals.get("workload") != workload_name:
+        return None
     if vals.get("kernel_sources_sha256_16") != kernel_sources_hash():
         return None
     try:
@@ -296,6 +321,115 @@ def time_adamw_lane(w, dev, steps, peaks, world):
             "unit": "GB/s", "frac": round(gbs / peak, 4) if peak else None, "bytes_per_element": 26}
 
 
+def make_step(w, dev, args):
+    """Seeded inputs of workload w, resident in HBM, and one step over them.
+    Returns (step, inputs) where inputs holds the tensors and byte counts."""
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+    mo.muon_reset_config()
+    inp = {}
+    if w.full_step:
+        params = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=dev) for i in range(w.count)]
+        grads = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev) for i in range(w.count)]
+        moms = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
+        mo.muon_set_config(mode=args.form, soft_threshold=args.soft_threshold)
+
+        def step():
+            mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
+        inp.update(params=params, grads=grads, moms=moms)
+        inp["bytes_in"] = sum(g.numel() * g.element_size() for g in grads)
+        inp["resident"] = inp["bytes_in"] + sum(p.numel() * p.element_size() for p in params) + \
+            sum(m.numel() * m.element_size() for m in moms)
+    else:
+        # NS-only workloads: one batched orthogonalisation per distinct shape,
+        # in place.  Every timed step re-orthogonalises the previous step's
+        # output (the work does not depend on the values; the input is
+        # normalised first), so no copy runs inside the timed region.
+        by_shape = {}
+        for i, s in enumerate(w.shapes):
+            by_shape.setdefault(s, []).append(i)
+        work = {s: torch.stack([wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev, dtype="bf16")
+                                for i in idx]) for s, idx in by_shape.items()}
+
+        def step():
+            for s in work:
+                mo.muon_orthogonalize(work[s], steps=5, mode=args.form)
+        inp["work"] = work
+        inp["bytes_in"] = sum(t.numel() * t.element_size() for t in work.values())
+        inp["resident"] = inp["bytes_in"]
+    return step, inp
+
+
+def device_time(step, steps, world, dev):
+    """ms of `steps` steps on the launching stream (CUDA events, barrier and
+    synchronize on both sides), max over ranks."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    return max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+
+
+def gemm_roofline(prof, ms_total, ms_per_step, peaks, peak_src, traffic):
+    gemm = prof.get("gemm_tc", {})
+    gemm_tf = (gemm["flops"] / (gemm["total_ms"] * 1e-3) / 1e12) if gemm.get("total_ms") else 0.0
+    # A kernel inside a long step runs at the power-capped sustained clock;
+    # one inside a short step at the burst clock.
+    long_step = ms_per_step >= 50.0
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    peak_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak_tf = peak_sust if long_step else peak_burst
+    launches = gemm.get("launches", 0)
+    return {
+        "kernel": "gemm_tc (tcgen05 grouped GEMM, all Newton-Schulz products)",
+        "bound": "tensor", "achieved": round(gemm_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
+        "frac": round(gemm_tf / peak_tf, 4) if peak_tf else None,
+        "traffic": traffic,
+        "peak_source": (f"{peak_src} bf16_tflops_sustained (step >= 50 ms)" if long_step else
+                        f"{peak_src} bf16_tflops (burst; step < 50 ms)") +
+                       "; fp16 operands run at the bf16 rate",
+        "frac_of_burst": round(gemm_tf / peak_burst, 4) if peak_burst else None,
+        "frac_of_sustained": round(gemm_tf / peak_sust, 4) if peak_sust else None,
+        "launches": launches,
+        "flops_per_launch": (gemm["flops"] / launches) if launches else None,
+        "avg_launch_ms": (gemm["total_ms"] / launches) if launches else None,
+        "share_of_step": round(gemm.get("total_ms", 0) / ms_total, 4) if ms_total else None,
+    }
+
+
+def measure_extra(w, dev, args, peaks, peak_src, world):
+    """Device-timed step of another workload (no e2e, no CPU leg)."""
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+    step, inp = make_step(w, dev, args)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    mo.muon_profile_reset()
+    mo.muon_profile_enable(True)
+    ms_total = device_time(step, args.steps, world, dev)
+    prof = mo.muon_profile_read()
+    mo.muon_profile_enable(False)
+    st, bad = mo.muon_device_status()
+    if st != mo.MUON_OK:
+        raise SystemExit(f"device status {mo.STATUS_NAMES.get(st, st)} (matrix {bad})")
+    ms = ms_total / args.steps
+    out = {"workload": w.name, "workload_id": w.wid, "matrices": w.count, "elements": w.elements,
+           "ms_per_step": round(ms, 4), "steps": args.steps,
+           "roofline": gemm_roofline(prof, ms_total, ms, peaks, peak_src, traffic_from_profiles(w.name))}
+    del step, inp
+    torch.cuda.empty_cache()
+    mo.muon_release_workspace()
+    return out
+
+
 def run_ours(args):
     import torch
     import matrix_orthogonalizing_optimizer_step_b200 as mo
@@ -310,34 +444,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
 
     # ---- inputs (seeded, resident in HBM) --------------------------------
-    if w.full_step:
-        params = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=dev) for i in range(w.count)]
-        grads = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev) for i in range(w.count)]
-        moms = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
-        mo.muon_reset_config()
-        mo.muon_set_config(mode=args.form, soft_threshold=args.soft_threshold)
-
-        def step():
-            mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
-        bytes_in = sum(g.numel() * g.element_size() for g in grads)
-        in_bytes_resident = bytes_in + sum(p.numel() * p.element_size() for p in params) + \
-            sum(m.numel() * m.element_size() for m in moms)
-    else:
-        # NS-only workloads: one batched orthogonalisation per distinct shape
-        by_shape = {}
-        for i, s in enumerate(w.shapes):
-            by_shape.setdefault(s, []).append(i)
-        src = {s: torch.stack([wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev, dtype="bf16")
-                               for i in idx]) for s, idx in by_shape.items()}
-        work = {s: t.clone() for s, t in src.items()}
-
-        def step():
-            for s in work:
-                work[s].copy_(src[s])
-                mo.muon_orthogonalize(work[s], steps=5, mode=args.form)
-        bytes_in = sum(t.numel() * t.element_size() for t in src.values())
-        in_bytes_resident = 2 * bytes_in
-
+    step, inp = make_step(w, dev, args)
     torch.cuda.synchronize()
     for _ in range(max(args.warmup, 3)):
         step()
@@ -355,22 +462,11 @@ def run_ours(args):
     mo.muon_profile_reset()
     mo.muon_profile_enable(True)
     launches0 = mo.muon_launch_count()
-    stream = torch.cuda.current_stream(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, dev)
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world, dev)
+    ms_total = device_time(step, args.steps, world, dev)
     launches = mo.muon_launch_count() - launches0
     prof = mo.muon_profile_read()
     mo.muon_profile_enable(False)
     clk = clocks.stop()
-    ms_total = ev0.elapsed_time(ev1)
-    ms_total = max_over_ranks(ms_total, world, dev)
     ms_per_step = ms_total / args.steps
 
     st, bad = mo.muon_device_status()
@@ -380,27 +476,7 @@ def run_ours(args):
     # ---- roofline of the dominant kernel -------------------------------------
     gemm = prof.get("gemm_tc", {})
     momk = prof.get("momentum_norm", {})
-    gemm_tf = (gemm["flops"] / (gemm["total_ms"] * 1e-3) / 1e12) if gemm.get("total_ms") else 0.0
-    # A kernel inside a long step runs at the power-capped sustained clock;
-    # one inside a short step at the burst clock.
-    long_step = ms_per_step >= 50.0
-    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    peak_sust = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    peak_tf = peak_sust if long_step else peak_burst
-    traffic = traffic_from_profiles()
-    roofline = {
-        "kernel": "gemm_tc (tcgen05 grouped GEMM, all Newton-Schulz products)",
-        "bound": "tensor", "achieved": round(gemm_tf, 2), "peak": peak_tf, "unit": "TFLOP/s",
-        "frac": round(gemm_tf / peak_tf, 4) if peak_tf else None,
-        "traffic": traffic,
-        "peak_source": (f"{peak_src} bf16_tflops_sustained (step >= 50 ms)" if long_step else
-                        f"{peak_src} bf16_tflops (burst; step < 50 ms)") +
-                       "; fp16 operands run at the bf16 rate",
-        "frac_of_burst": round(gemm_tf / peak_burst, 4) if peak_burst else None,
-        "frac_of_sustained": round(gemm_tf / peak_sust, 4) if peak_sust else None,
-        "launches": gemm.get("launches", 0), "avg_launch_ms": (gemm["total_ms"] / gemm["launches"]) if gemm.get("launches") else None,
-        "share_of_step": round(gemm.get("total_ms", 0) / ms_total, 4) if ms_total else None,
-    }
+    roofline = gemm_roofline(prof, ms_total, ms_per_step, peaks, peak_src, traffic_from_profiles(w.name))
     mom_gbs = (momk["bytes"] / (momk["total_ms"] * 1e-3) / 1e9) if momk.get("total_ms") else 0.0
     peak_gbs = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     roofline_mom = {
@@ -421,6 +497,7 @@ def run_ours(args):
     if not args.no_e2e:
         e2e_steps = max(1, min(args.steps, 10))
         if w.full_step:
+            params, grads = inp["params"], inp["grads"]
             host_g = [g.detach().to("cpu").pin_memory() for g in grads]
             host_p = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
 
@@ -430,37 +507,48 @@ def run_ours(args):
                 step()
                 for h, p in zip(host_p, params):
                     h.copy_(p, non_blocking=True)
-            h2d = bytes_in
+            h2d = inp["bytes_in"]
             d2h = sum(p.numel() * p.element_size() for p in params)
+            note = "pinned host grads -> HBM, muon_step, params -> pinned host, per step"
         else:
-            host_in = {s: t.detach().to("cpu").pin_memory() for s, t in src.items()}
-            host_out = {s: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for s, t in src.items()}
+            work = inp["work"]
+            host_in = {s: t.detach().to("cpu").pin_memory() for s, t in work.items()}
+            host_out = {s: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for s, t in work.items()}
 
             def e2e_step():
                 for s in work:
                     work[s].copy_(host_in[s], non_blocking=True)
                     mo.muon_orthogonalize(work[s], steps=5, mode=args.form)
                     host_out[s].copy_(work[s], non_blocking=True)
-            h2d = bytes_in
-            d2h = bytes_in
+            h2d = inp["bytes_in"]
+            d2h = inp["bytes_in"]
+            note = "pinned host matrices -> HBM, muon_orthogonalize, results -> pinned host, per step"
         e2e_step()
         torch.cuda.synchronize()
-        barrier(world, dev)
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / e2e_steps
+        e2e_ms = device_time(e2e_step, e2e_steps, world, dev) / e2e_steps
         e2e = {"value": round(e2e_ms, 4), "unit": "ms", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": e2e_steps,
-               "note": "pinned host grads -> HBM, muon_step, params -> pinned host, per step"}
+               "d2h_bytes_per_step": int(d2h), "steps": e2e_steps, "note": note}
+        del e2e_step
+        if w.full_step:
+            del host_g, host_p
+        else:
+            del host_in, host_out
+
+    resident_mb = inp["resident"] / 1e6
+    del step, inp
+    torch.cuda.empty_cache()
+    mo.muon_release_workspace()
 
     # ---- the hybrid optimizer's AdamW lane on the model's AdamW parameters ----
     adamw = None
     if w.adamw_numels and not args.no_adamw:
         adamw = time_adamw_lane(w, dev, max(args.steps, 5), peaks, world)
+
+    # ---- other workloads, device-timed (extra keys) ----------------------------
+    extra = {}
+    for wid in [int(x) for x in args.also.split(",") if x.strip() and int(x) != w.wid]:
+        ew = wl.WORKLOADS[wid]
+        extra[ew.name] = measure_extra(ew, dev, args, peaks, peak_src, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -479,7 +567,7 @@ def run_ours(args):
                        "coeffs": [3.4445, -4.775, 2.0315], "momentum": 0.95, "nesterov": True,
                        "lr": 6e-4, "momentum_dtype": w.momentum_dtype, "param_dtype": w.param_dtype,
                        "soft_threshold": args.soft_threshold,
-                       "l2": f"inputs larger than L2: {in_bytes_resident / 1e6:.0f} MB read per step",
+                       "l2": f"inputs larger than L2: {resident_mb:.0f} MB read per step",
                        "parallelism": f"replica x{world} (independent per GPU)"},
             "ns_tflops_per_step": round(ns_tflops, 2),
             "ns_tflops_standard_equivalent": round(ns_tflops_std, 2),
@@ -487,6 +575,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
             "adamw_lane": adamw,
+            "also": extra,
         }
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -495,20 +584,39 @@ def run_ours(args):
 
 
 def run_reference(args):
+    """The oracle arm: the fp64 CPU oracle, as it stands, on the host cores.
+    Each step is a bounded sample of the workload: one matrix, taken from the
+    distinct shapes in rotation (and from the matrices of a shape in order),
+    so K steps sample every shape about K / shapes times.  The reported step
+    time is the per-shape mean oracle time x that shape's count, summed: an
+    extrapolation to the whole step of the workload.  Warm-up steps run the
+    cheapest shape's first matrix."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    from oracle import muon_oracle as orc
     w = wl.WORKLOADS[args.workload]
-    budget = max(1.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    groups = _distinct_shapes(w)
+    cheapest = min(groups, key=lambda g: orc.ns_flops(min(g[0]), max(g[0]), 5, "standard"))[1][0]
     for _ in range(args.warmup):
-        cpu_oracle_step_ms(w, budget, args.form, args.soft_threshold)
-    vals = []
-    cores, sample = None, None
-    for _ in range(args.steps):
-        v, cores, sample = cpu_oracle_step_ms(w, budget, args.form, args.soft_threshold)
-        vals.append(v)
-    value = statistics.fmean(vals)
+        _oracle_seconds(w, cheapest, args.form, args.soft_threshold)
+    per_shape = {}
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        s, idx = groups[k % len(groups)]
+        i = idx[(k // len(groups)) % len(idx)]
+        per_shape.setdefault(s, []).append(_oracle_seconds(w, i, args.form, args.soft_threshold))
+    # a run with fewer steps than shapes still needs every shape once
+    for s, idx in groups:
+        if s not in per_shape:
+            per_shape[s] = [_oracle_seconds(w, idx[0], args.form, args.soft_threshold)]
+    wall = time.perf_counter() - t0
+    value = _extrapolate_ms(w, per_shape)
+    cores = _host_cores()
+    sample = (f"{sum(len(v) for v in per_shape.values())} single-matrix samples over {len(groups)} shapes "
+              f"(one matrix per step, shapes in rotation; {wall:.1f} s of oracle time), fp64 NumPy oracle, "
+              f"per-shape mean time x count (extrapolated to the whole step of {w.count} matrices)")
     out = {
         "impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "ms",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -13,9 +13,13 @@ momentum read per step), far larger than the 126 MB L2, so no flush is
 needed between steps.  A short device-timed measurement of the GPT-2 124M
 set follows as an extra key (--also 0 turns it off).
 
-Prints ONE JSON line on rank 0.  Under torchrun each rank runs its own
-replica of the workload (weak scaling, no data-path collective) and the
-device time is the max over ranks.
+Prints ONE JSON line on rank 0.  Under torchrun (N > 1) the ranks share
+ONE step of the workload (strong scaling): each rank runs the library's step
+on the whole matrices it owns (longest-processing-time partition on the
+Newton-Schulz FLOPs) and one in-place all-gather per dtype spreads the
+updated parameters (sharded.py).  --replicas runs an independent replica per
+GPU instead (weak scaling, no data-path collective).  The device time is the
+max over ranks.
 """
 from __future__ import annotations
 
@@ -52,6 +56,8 @@ def parse():
                     help="skip the AdamW-lane measurement on the model's AdamW parameters")
     ap.add_argument("--soft-threshold", type=float, default=0.0,
                     help="lam of the soft-threshold split of the update (0 = plain Muon)")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with N > 1: one independent replica of the workload per GPU instead of the sharded step")
     ap.add_argument("--also", default="2",
                     help="comma-separated workload ids timed on the device after the main one (extra key)")
     ap.add_argument("--subset", type=int, default=0,
@@ -321,9 +327,11 @@ def time_adamw_lane(w, dev, steps, peaks, world):
             "unit": "GB/s", "frac": round(gbs / peak, 4) if peak else None, "bytes_per_element": 26}
 
 
-def make_step(w, dev, args):
+def make_step(w, dev, args, sharded_over=1):
     """Seeded inputs of workload w, resident in HBM, and one step over them.
-    Returns (step, inputs) where inputs holds the tensors and byte counts."""
+    Returns (step, inputs) where inputs holds the tensors and byte counts.
+    sharded_over > 1: the step is the sharded step over that many ranks
+    (whole matrices per rank, then one all-gather of the parameters)."""
     import torch
     import matrix_orthogonalizing_optimizer_step_b200 as mo
     mo.muon_reset_config()
@@ -334,8 +342,16 @@ def make_step(w, dev, args):
         moms = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
         mo.muon_set_config(mode=args.form, soft_threshold=args.soft_threshold)
 
-        def step():
-            mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
+        if sharded_over > 1:
+            from matrix_orthogonalizing_optimizer_step_b200 import sharded
+            owner = sharded.partition([tuple(p.shape) for p in params], sharded_over)
+            inp["owner"] = owner
+
+            def step():
+                sharded.sharded_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4, owner=owner)
+        else:
+            def step():
+                mo.muon_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4)
         inp.update(params=params, grads=grads, moms=moms)
         inp["bytes_in"] = sum(g.numel() * g.element_size() for g in grads)
         inp["resident"] = inp["bytes_in"] + sum(p.numel() * p.element_size() for p in params) + \
@@ -444,7 +460,10 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
 
     # ---- inputs (seeded, resident in HBM) --------------------------------
-    step, inp = make_step(w, dev, args)
+    # N > 1: the sharded step of ONE workload over all ranks (strong scaling),
+    # unless --replicas asks for one independent replica per GPU (weak)
+    shard = world > 1 and not args.replicas and w.full_step
+    step, inp = make_step(w, dev, args, sharded_over=world if shard else 1)
     torch.cuda.synchronize()
     for _ in range(max(args.warmup, 3)):
         step()
@@ -546,7 +565,8 @@ def run_ours(args):
 
     # ---- other workloads, device-timed (extra keys) ----------------------------
     extra = {}
-    for wid in [int(x) for x in args.also.split(",") if x.strip() and int(x) != w.wid]:
+    also = [int(x) for x in args.also.split(",") if x.strip() and int(x) != w.wid] if world == 1 else []
+    for wid in also:
         ew = wl.WORKLOADS[wid]
         extra[ew.name] = measure_extra(ew, dev, args, peaks, peak_src, world)
 
@@ -560,7 +580,7 @@ def run_ours(args):
             "metric": METRIC, "value": round(ms_per_step, 4), "unit": "ms",
             "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
             "ms_per_step": round(ms_per_step, 4), "higher_is_better": False,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if shard else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; shapes of the named model family, random values)",
             "config": {"workload": w.name, "workload_id": w.wid, "matrices": w.count,
                        "elements": w.elements, "ns_steps": 5, "ns_form": args.form,
@@ -568,7 +588,9 @@ def run_ours(args):
                        "lr": 6e-4, "momentum_dtype": w.momentum_dtype, "param_dtype": w.param_dtype,
                        "soft_threshold": args.soft_threshold,
                        "l2": f"inputs larger than L2: {resident_mb:.0f} MB read per step",
-                       "parallelism": f"replica x{world} (independent per GPU)"},
+                       "parallelism": (f"sharded x{world} (whole matrices per rank, LPT on Newton-Schulz "
+                                       f"FLOPs; one all-gather of the parameters per step)") if shard else
+                                      f"replica x{world} (independent per GPU)"},
             "ns_tflops_per_step": round(ns_tflops, 2),
             "ns_tflops_standard_equivalent": round(ns_tflops_std, 2),
             "roofline": roofline, "roofline_momentum": roofline_mom,

@@ -29,9 +29,28 @@
  *    except muon_device_status and muon_profile_read.
  *  - The library owns a cached device workspace sized for the last shape set
  *    (released by muon_release_workspace or at unload).  Calls are not
- *    thread-safe; use one thread per library instance.
+ *    thread-safe; use one thread per library instance.  Calls may switch
+ *    streams: a call's use of the workspace is ordered after the previous
+ *    call's, on whichever stream that ran (an event wait, not a host sync).
+ *    The caller's own tensors are not synchronised across streams.
  *  - Every call returns a status (< 0 on error) and never throws.  On an
  *    argument error nothing is enqueued; muon_last_error() describes it.
+ *  - Every device-side wait (a CTA pair waiting for its operands, for another
+ *    tile's results, or for its accumulator) is bounded: after the limit the
+ *    kernel records MUON_ERR_TIMEOUT in the device status word, drains its own
+ *    copies and tensor-core work, frees its tensor memory and exits.
+ *  - Environment knobs, read when a plan is built (tests and debugging):
+ *    MUON_WAIT_LIMIT_MS  bound of every device-side wait (1..10000, default 1000)
+ *    MUON_FAULT          alloc | launch | timeout: fail the workspace
+ *                        allocation (MUON_ERR_NO_MEMORY) or the first launch
+ *                        (MUON_ERR_CUDA) of a call before anything is
+ *                        enqueued, or give the first tile of a chained launch
+ *                        a dependency that is never met (MUON_ERR_TIMEOUT
+ *                        after the wait limit)
+ *    MUON_CHAIN_LAUNCH / MUON_SLOT_LAUNCHES  force one launch for the whole
+ *                        Newton-Schulz chain / one launch per chain slot
+ *    MUON_TMA_STORE=0    plain per-lane stores in the GEMM epilogue
+ *    MUON_PROFILE_VERBOSE  print every traced launch to stderr
  */
 #ifndef MUON_B200_H
 #define MUON_B200_H
@@ -136,7 +155,7 @@ MUON_API int muon_device_status(int* bad_index);
  * steps   T in 0..MUON_MAX_STEPS; 0 returns the normalised X
  * mode    MUON_NS_STANDARD | MUON_NS_GRAM | MUON_NS_AUTO, optionally | MUON_PREC_FP32
  * eps and the Gram restart schedule come from the installed config.
- * A zero matrix returns zeros.
+ * A zero matrix returns zeros (also with eps = 0).
  */
 MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* coeffs, int steps, int mode);
 
@@ -151,8 +170,11 @@ MUON_API int muon_orthogonalize(int batch, int m, int n, void* X, const float* c
  * shape_list  host int[2*count]: rows_i, cols_i of parameter i (>= 1)
  * With muon_config.soft_threshold = lam > 0, U is first clipped elementwise
  * to [-lam/2, lam/2] (its soft-thresholded outlier part is dropped; M keeps
- * it).  Coefficients, steps, NS form, restarts, eps, dtypes and the
- * threshold come from the installed config.  16-byte aligned pointers and
+ * it).  Coefficients and steps come from the shape's registered schedule
+ * (muon_set_shape_coeffs) or else from the installed config; NS form,
+ * restarts, eps, dtypes and the threshold from the installed config.  A
+ * matrix whose U is zero (e.g. an expert that received no tokens) leaves its
+ * parameter unchanged, also with eps = 0.  16-byte aligned pointers and
  * cols % 8 == 0 take the vectorised paths (otherwise element-wise ones).
  * Distinct parameters must not overlap.
  */
@@ -181,6 +203,63 @@ MUON_API int muon_adamw_step(void* const* params, const void* const* grads, void
                              void* const* exp_avg_sq, const long long* numels, int count, float lr, float beta1,
                              float beta2, float eps, float weight_decay, int step);
 
+/*
+ * muon_hybrid_step -- the whole hybrid optimizer step of a model: muon_step
+ * over its 2-D hidden matrices and the AdamW step (as muon_adamw_step) over
+ * the rest, with the AdamW lane's elements in the SAME grouped elementwise
+ * launch as the Muon momentum pass (its chunks follow the Muon chunks in one
+ * grid), followed by the Newton-Schulz launches.
+ *   [NanoGPT-Muon] "从 SGD 到 Muon" (Muon for the 2-D hidden weights, AdamW
+ *   for embeddings, the output head and 1-D parameters), "工程复现清单".
+ * The Muon arguments are muon_step's; `adamw` describes the AdamW lane (host
+ * struct, read during the call; its arrays as in muon_adamw_step).  Both lanes
+ * use the installed config's param_dtype and grad_dtype.  Every argument of
+ * both lanes is checked before anything is enqueued.  Results equal a
+ * muon_step followed by a muon_adamw_step with the same arguments.
+ */
+typedef struct muon_adamw_lane {
+    void* const* params;           /* count device pointers, updated in place      */
+    const void* const* grads;      /* count device pointers, read only             */
+    void* const* exp_avg;          /* count device pointers, fp32, updated         */
+    void* const* exp_avg_sq;       /* count device pointers, fp32, updated         */
+    const long long* numels;       /* count element counts (>= 1)                  */
+    int count;                     /* >= 1                                          */
+    float lr, beta1, beta2, eps, weight_decay;
+    int step;                      /* >= 1, for the bias corrections               */
+} muon_adamw_lane;
+
+MUON_API int muon_hybrid_step(void* const* params, const void* const* grads, void* const* momentum, float mu,
+                              int nesterov, float lr, const int* shape_list, int count,
+                              const muon_adamw_lane* adamw);
+
+/* ---- per-shape coefficient schedules ----------------------------------------
+ *
+ * [ROOT] (staging.reportify.cn tag page, "ROOT优化器的技术创新"): the quintic
+ * Newton-Schulz coefficients are adapted to each matrix size (m, n) instead of
+ * one fixed set for all shapes ("现有优化器的核心局限": a fixed set leaves a
+ * shape-dependent orthogonalisation error).  A schedule is one (a, b, c)
+ * triple per step; matrices of different shapes in ONE muon_step each run
+ * their own schedule inside the same grouped launches.
+ *
+ * muon_set_shape_coeffs -- register the schedule of muon_step for matrices of
+ * rows x cols.  A matrix and its transpose share one entry (the key is the
+ * short and the long side).  coeffs: host array of 3*steps floats, (a, b, c) of
+ * step k at [3k..3k+2], copied; steps in 0..MUON_MAX_STEPS (0: the matrix is
+ * only normalised).  Re-registering a shape replaces its schedule.  Matrices
+ * whose shape has no entry use muon_config.coeffs / muon_config.steps.
+ * MUON_ERR_INVALID_ARG for sizes < 1, steps out of range, NULL or non-finite
+ * coeffs, or more than MUON_MAX_SHAPE_SCHEDULES shapes.  Host-only: enqueues
+ * nothing.  muon_orthogonalize is unaffected (it takes its coefficients as an
+ * argument).
+ * muon_get_shape_coeffs -- *steps = the registered step count (-1 if the shape
+ * has none) and, if coeffs is not NULL, the 3 * steps coefficients.
+ * muon_clear_shape_coeffs -- remove every entry.
+ */
+#define MUON_MAX_SHAPE_SCHEDULES 64
+MUON_API int muon_set_shape_coeffs(int rows, int cols, const float* coeffs, int steps);
+MUON_API int muon_get_shape_coeffs(int rows, int cols, float* coeffs, int* steps);
+MUON_API int muon_clear_shape_coeffs(void);
+
 /* ---- allocation-free normalisation ---------------------------------------
  *
  * The pages have no counterpart to this call: it exists for callers that
@@ -208,7 +287,9 @@ MUON_API int muon_adamw_step(void* const* params, const void* const* grads, void
  * shares the array and it keeps the last call's contents: each call clears
  * the counters it uses, and calls that overlap on the GPU (other streams,
  * other threads) race on it.  A matrix whose norm is not finite leaves its Y
- * untouched.
+ * untouched; a zero matrix gives a zero Y, also with eps = 0.  The device
+ * addresses found at set-up are cached per device without a lock, like the
+ * rest of the library's state (calls are not thread-safe).
  */
 #define MUON_NOALLOC_MAX_MATRICES 1024
 #define MUON_NOALLOC_MAX_CHUNKS 65536 /* chunks of 8192 elements: 512 Mi elements in one call */

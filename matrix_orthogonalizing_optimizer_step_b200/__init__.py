@@ -14,7 +14,7 @@ from . import _lib
 from ._lib import (  # noqa: F401
     MUON_DTYPE_BF16, MUON_DTYPE_F32, MUON_ERR_CUDA, MUON_ERR_INVALID_ARG,
     MUON_ERR_NO_MEMORY, MUON_ERR_NONFINITE, MUON_ERR_TIMEOUT,
-    MUON_ERR_UNSUPPORTED, MUON_MAX_STEPS, MUON_NS_AUTO, MUON_NS_GRAM,
+    MUON_ERR_UNSUPPORTED, MUON_MAX_SHAPE_SCHEDULES, MUON_MAX_STEPS, MUON_NS_AUTO, MUON_NS_GRAM,
     MUON_NS_STANDARD, MUON_OK, MUON_PREC_FP32, STATUS_NAMES,
 )
 
@@ -93,11 +93,7 @@ def muon_orthogonalize(X, coeffs=TUNED_COEFFS, steps=5, mode="auto", fp32=False)
     return X
 
 
-def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
-    """One Muon step over lists of 2D CUDA tensors (updated in place).
-
-    grads, momentum and params use the installed config's dtypes.
-    """
+def _muon_lane(params, grads, momentum):
     count = len(params)
     if not (len(grads) == len(momentum) == count) or count == 0:
         raise ValueError("params, grads and momentum must be non-empty lists of equal length")
@@ -113,15 +109,10 @@ def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
             raise ValueError("tensors must be contiguous")
         shapes.extend(p.shape)
     S = (ctypes.c_int * len(shapes))(*shapes)
-    _bind_stream(params[0].device)
-    _check(lib().muon_step(P, G, M, float(mu), 1 if nesterov else 0, float(lr), S, count))
+    return P, G, M, S, count
 
 
-def muon_adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
-                    weight_decay=0.1):
-    """AdamW step (the hybrid optimizer's lane for embeddings, head and 1-D
-    parameters) over lists of CUDA tensors, updated in place.  Moments are
-    fp32; params and grads use the installed config's dtypes."""
+def _adamw_lane(params, grads, exp_avg, exp_avg_sq):
     count = len(params)
     if not (len(grads) == len(exp_avg) == len(exp_avg_sq) == count) or count == 0:
         raise ValueError("params, grads, exp_avg and exp_avg_sq must be non-empty lists of equal length")
@@ -131,10 +122,43 @@ def muon_adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=6e-4, betas=(0.
     vp = ctypes.c_void_p
     arr = lambda ts: (vp * count)(*[t.data_ptr() for t in ts])  # noqa: E731
     N = (ctypes.c_longlong * count)(*[t.numel() for t in params])
+    return arr(params), arr(grads), arr(exp_avg), arr(exp_avg_sq), N, count
+
+
+def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
+    """One Muon step over lists of 2D CUDA tensors (updated in place).
+
+    grads, momentum and params use the installed config's dtypes.
+    """
+    P, G, M, S, count = _muon_lane(params, grads, momentum)
     _bind_stream(params[0].device)
-    _check(lib().muon_adamw_step(arr(params), arr(grads), arr(exp_avg), arr(exp_avg_sq), N, count,
-                                 float(lr), float(betas[0]), float(betas[1]), float(eps),
-                                 float(weight_decay), int(step)))
+    _check(lib().muon_step(P, G, M, float(mu), 1 if nesterov else 0, float(lr), S, count))
+
+
+def muon_hybrid_step(params, grads, momentum, adam_params, adam_grads, exp_avg, exp_avg_sq, step,
+                     mu=0.95, nesterov=True, lr=6e-4, adam_lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
+                     weight_decay=0.1):
+    """The hybrid step in one elementwise launch plus the Newton-Schulz
+    launches: muon_step over (params, grads, momentum) and the AdamW step over
+    the adam_* lists (fp32 moments), as muon_step + muon_adamw_step."""
+    P, G, M, S, count = _muon_lane(params, grads, momentum)
+    AP, AG, AM, AV, N, acount = _adamw_lane(adam_params, adam_grads, exp_avg, exp_avg_sq)
+    lane = _lib.MuonAdamwLane(AP, AG, AM, AV, N, acount, float(adam_lr), float(betas[0]), float(betas[1]),
+                              float(eps), float(weight_decay), int(step))
+    _bind_stream(params[0].device)
+    _check(lib().muon_hybrid_step(P, G, M, float(mu), 1 if nesterov else 0, float(lr), S, count,
+                                  ctypes.byref(lane)))
+
+
+def muon_adamw_step(params, grads, exp_avg, exp_avg_sq, step, lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
+                    weight_decay=0.1):
+    """AdamW step (the hybrid optimizer's lane for embeddings, head and 1-D
+    parameters) over lists of CUDA tensors, updated in place.  Moments are
+    fp32; params and grads use the installed config's dtypes."""
+    AP, AG, AM, AV, N, count = _adamw_lane(params, grads, exp_avg, exp_avg_sq)
+    _bind_stream(params[0].device)
+    _check(lib().muon_adamw_step(AP, AG, AM, AV, N, count, float(lr), float(betas[0]), float(betas[1]),
+                                 float(eps), float(weight_decay), int(step)))
 
 
 def muon_default_config():
@@ -189,9 +213,37 @@ def muon_set_config(steps=None, coeffs=None, mode=None, restart_mask=None,
 
 
 def muon_reset_config():
+    """Install the default config and remove every per-shape schedule."""
     cfg = _lib.MuonConfig()
     _check(lib().muon_default_config(ctypes.byref(cfg)))
     _check(lib().muon_set_config(ctypes.byref(cfg)))
+    _check(lib().muon_clear_shape_coeffs())
+
+
+def muon_set_shape_coeffs(rows, cols, coeffs):
+    """Register the Newton-Schulz schedule of muon_step for rows x cols
+    matrices (and their transposes): a list of (a, b, c) triples, one per
+    step (an empty list: normalisation only)."""
+    triples = [tuple(float(x) for x in t) for t in coeffs]
+    if any(len(t) != 3 for t in triples):
+        raise ValueError("coeffs must be (a, b, c) triples")
+    flat = [x for t in triples for x in t]
+    arr = (ctypes.c_float * max(len(flat), 1))(*flat)
+    _check(lib().muon_set_shape_coeffs(int(rows), int(cols), arr, len(triples)))
+
+
+def muon_get_shape_coeffs(rows, cols):
+    """The registered schedule of rows x cols matrices, or None."""
+    arr = (ctypes.c_float * (3 * MUON_MAX_STEPS))()
+    steps = ctypes.c_int(-1)
+    _check(lib().muon_get_shape_coeffs(int(rows), int(cols), arr, ctypes.byref(steps)))
+    if steps.value < 0:
+        return None
+    return [tuple(arr[3 * k:3 * k + 3]) for k in range(steps.value)]
+
+
+def muon_clear_shape_coeffs():
+    _check(lib().muon_clear_shape_coeffs())
 
 
 def muon_device_status(device=None):

@@ -24,6 +24,7 @@ MUON_DTYPE_BF16 = 0
 MUON_DTYPE_F32 = 1
 
 MUON_MAX_STEPS = 16
+MUON_MAX_SHAPE_SCHEDULES = 64
 
 STATUS_NAMES = {
     MUON_OK: "MUON_OK", MUON_ERR_INVALID_ARG: "MUON_ERR_INVALID_ARG",
@@ -39,6 +40,8 @@ EXPORTS = (
     "muon_device_status", "muon_orthogonalize", "muon_step",
     "muon_profile_enable", "muon_profile_read", "muon_profile_reset",
     "muon_launch_count", "muon_normalize_noalloc", "muon_adamw_step",
+    "muon_set_shape_coeffs", "muon_get_shape_coeffs", "muon_clear_shape_coeffs",
+    "muon_hybrid_step",
 )
 
 
@@ -53,6 +56,23 @@ class MuonConfig(ctypes.Structure):
         ("param_dtype", ctypes.c_int),
         ("grad_dtype", ctypes.c_int),
         ("soft_threshold", ctypes.c_float),
+    ]
+
+
+class MuonAdamwLane(ctypes.Structure):
+    _fields_ = [
+        ("params", ctypes.POINTER(ctypes.c_void_p)),
+        ("grads", ctypes.POINTER(ctypes.c_void_p)),
+        ("exp_avg", ctypes.POINTER(ctypes.c_void_p)),
+        ("exp_avg_sq", ctypes.POINTER(ctypes.c_void_p)),
+        ("numels", ctypes.POINTER(ctypes.c_longlong)),
+        ("count", ctypes.c_int),
+        ("lr", ctypes.c_float),
+        ("beta1", ctypes.c_float),
+        ("beta2", ctypes.c_float),
+        ("eps", ctypes.c_float),
+        ("weight_decay", ctypes.c_float),
+        ("step", ctypes.c_int),
     ]
 
 
@@ -104,6 +124,11 @@ def load(path=LIB_PATH):
         "muon_adamw_step": (c_int, [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
                                     ctypes.POINTER(vp), ctypes.POINTER(ctypes.c_longlong), c_int,
                                     c_float, c_float, c_float, c_float, c_float, c_int]),
+        "muon_set_shape_coeffs": (c_int, [c_int, c_int, ctypes.POINTER(c_float), c_int]),
+        "muon_get_shape_coeffs": (c_int, [c_int, c_int, ctypes.POINTER(c_float), ctypes.POINTER(c_int)]),
+        "muon_clear_shape_coeffs": (c_int, []),
+        "muon_hybrid_step": (c_int, [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), c_float, c_int,
+                                     c_float, ctypes.POINTER(c_int), c_int, ctypes.POINTER(MuonAdamwLane)]),
     }
     assert set(sig) == set(EXPORTS)
     for name, (res, args) in sig.items():

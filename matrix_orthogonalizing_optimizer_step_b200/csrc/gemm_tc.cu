@@ -33,6 +33,14 @@
 // per-matrix completion counter; matrices progress independently, so the
 // dependency waits of one matrix are filled with other matrices' tiles.
 //
+// Tiles are claimed, in list order, from a global ticket by the leader CTA's
+// producer, one tile ahead of the one it is loading, and handed to every role
+// of both CTAs through a small ring of tile indices in shared memory.  A tile
+// that waits on earlier tiles therefore only ever waits on tiles that running
+// pairs have claimed: the launch makes progress however many of its pairs
+// are resident (other kernels may hold SMs), and the dynamic order also
+// balances tiles of unequal K across pairs.
+//
 // Every wait is bounded: on expiry the kernel records a timeout in the device
 // status word, drains its own copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -60,7 +68,11 @@ constexpr uint32_t TMEM_COLS = 512;  // 2 accumulators x 256 fp32 columns
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
 constexpr int STORE_BOX_BYTES = 64 * 32;  // one TMA store box: 32 rows of 64 bytes
 constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per epilogue warp
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 256 /*barriers*/;
+constexpr int SCHED = 8;  // depth of the tile-index ring
+// readers of every ring slot: the leader's MMA thread, the peer's producer,
+// and the epilogue warps of both CTAs
+constexpr uint32_t SCHED_READERS = 2 + 2 * EPI_WARPS;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 512 /*barriers, ring*/;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
 
 struct Shared {
@@ -68,10 +80,14 @@ struct Shared {
     uint64_t empty[STAGES];  // each CTA: its slot may be refilled (leader's MMA commit)
     uint64_t tfull[2];       // each CTA: accumulator ready (leader's MMA commit)
     uint64_t tempty[2];      // leader: all 2 x EPI_WARPS epilogue warps drained the accumulator
+    uint64_t sfull[SCHED];   // each CTA: ring slot holds a claimed tile index (leader's producer)
+    uint64_t sempty[SCHED];  // leader: every reader of both CTAs has read the ring slot
     uint64_t drain;
+    int sched[SCHED];        // claimed tile indices; ntiles: no more tiles
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Shared) <= 512, "barrier area");
 
 // Symmetric operands are stored as upper 256 x 256 tiles: the 64-wide K slice
 // kb of the 256-row block `blk` lies in a lower (unstored) tile when blk > kb/4.
@@ -101,8 +117,53 @@ __device__ __forceinline__ void record_timeout(Shared* sh, DeviceStatus* st) {
     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
 }
 
-__device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t rank, int pair, int npairs) {
+// Next unclaimed tile of the launch (ntiles once the list is exhausted).
+__device__ __forceinline__ int claim_tile(const TcLaunch& L) {
+    const unsigned t = atomicAdd(L.ticket, 1u);
+    return t < static_cast<unsigned>(L.ntiles) ? static_cast<int>(t) : L.ntiles;
+}
+
+// Writer side of the tile-index ring (the leader's producer): publish t in
+// the same slot of both CTAs' rings once every reader has read that slot's
+// previous value.  False when that wait ran out.
+struct RingWriter {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ bool push(Shared* sh, int t, volatile int* abort_flag, unsigned long long limit) {
+        if (!mbar_wait_cluster(&sh->sempty[slot], phase ^ 1u, abort_flag, limit)) return false;
+        const uint32_t v = smem_u32(&sh->sched[slot]), b = smem_u32(&sh->sfull[slot]);
+#pragma unroll
+        for (uint32_t r = 0; r < 2; ++r) {
+            st_shared_cluster_u32(map_to_cta(v, r), static_cast<uint32_t>(t));
+            mbar_arrive_cluster(map_to_cta(b, r));  // release: the index is visible first
+        }
+        if (++slot == SCHED) {
+            slot = 0;
+            phase ^= 1u;
+        }
+        return true;
+    }
+};
+
+// Reader side: the next published tile index, or -1 when the wait ran out.
+struct RingReader {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ int pop(Shared* sh, volatile int* abort_flag, unsigned long long limit) {
+        if (!mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit)) return -1;
+        const int t = *reinterpret_cast<volatile int*>(&sh->sched[slot]);
+        mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sempty[slot]), 0));  // read: the slot is free
+        if (++slot == SCHED) {
+            slot = 0;
+            phase ^= 1u;
+        }
+        return t;
+    }
+};
+
+__device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t rank) {
     volatile int* abort_flag = &sh->abort;
+    const unsigned long long lim = L.wait_ns;
     const bool leader = rank == 0;
     int stage = 0;
     uint32_t phase = 0;
@@ -110,20 +171,38 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     bool ok = true;
     int last_a = -1, last_b = -1;
     unsigned seen_mat = ~0u, seen_done = 0;  // counters only grow within a launch
-    // The next tile's record is fetched while the current tile runs, and its
-    // dependency and tensor maps are acquired right after the current tile's
-    // last fill is issued (the slices still queued in the ring hide the wait),
-    // so consecutive tiles follow each other without a gap in the fills.
+    RingWriter wr;
+    RingReader rd;
+    // The leader claims tiles and publishes them to both CTAs' rings; the
+    // peer reads them.  -1: a wait ran out.
+    auto next_tile = [&]() -> int {
+        if (leader) {
+            const int t = claim_tile(L);
+            return wr.push(sh, t, abort_flag, lim) ? t : -1;
+        }
+        return rd.pop(sh, abort_flag, lim);
+    };
+    // The next tile is claimed (and its record fetched) while the current one
+    // is loaded, and its dependency and tensor maps are acquired right after
+    // the current tile's last fill is issued (the slices still queued in the
+    // ring hide the wait), so consecutive tiles follow each other without a
+    // gap in the fills.
     bool early = false;  // the current tile's dependency was acquired early
+    int t = next_tile();
     TcTile nxt;
-    if (pair < L.ntiles) nxt = load_tile(L.tiles, pair);
-    for (int t = pair; t < L.ntiles && ok; t += npairs) {
+    if (t < 0) ok = false;
+    if (ok && t < L.ntiles) nxt = load_tile(L.tiles, t);
+    while (ok && t < L.ntiles) {
         const TcTile tile = nxt;
-        const int tn = t + npairs;
+        const int tn = next_tile();
+        if (tn < 0) {
+            ok = false;
+            break;
+        }
         if (tn < L.ntiles) nxt = load_tile(L.tiles, tn);
         // operands produced by earlier chain slots of the same matrix
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
-            if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag)) {
+            if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag, lim)) {
                 ok = false;
                 break;
             }
@@ -155,7 +234,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
         const int brow = bj * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows (N)
         const int nk = (K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
-            if (!mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag)) {
+            if (!mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag, lim)) {
                 ok = false;
                 break;
             }
@@ -202,6 +281,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 last_b = nxt.b_map;
             }
         }
+        t = tn;
     }
     if (!ok) record_timeout(sh, L.status);
     // Drain (leader): the last fills of every stage must have landed before
@@ -210,7 +290,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
         const uint32_t first = issued > STAGES ? issued - STAGES : 0;
         int never = 0;
         for (uint32_t i = first; i < issued; ++i) {
-            if (!mbar_wait(&sh->full[i % STAGES], (i / STAGES) & 1u, &never)) {
+            if (!mbar_wait(&sh->full[i % STAGES], (i / STAGES) & 1u, &never, lim)) {
                 atomicOr(&L.status->bits, ST_TIMEOUT);
                 break;
             }
@@ -218,9 +298,9 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     }
 }
 
-__device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base, int pair,
-                           int npairs) {
+__device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base) {
     volatile int* abort_flag = &sh->abort;
+    const unsigned long long lim = L.wait_ns;
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -228,11 +308,19 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     bool ok = true;
     bool issued_any = false;
     const uint32_t tiles_base = smem_u32(tiles_smem);
+    RingReader rd;
+    int t = rd.pop(sh, abort_flag, lim);
+    if (t < 0) ok = false;
     TcTile nxt;
-    if (pair < L.ntiles) nxt = load_tile(L.tiles, pair);
-    for (int t = pair; t < L.ntiles && ok; t += npairs) {
+    if (ok && t < L.ntiles) nxt = load_tile(L.tiles, t);
+    while (ok && t < L.ntiles) {
         const TcTile tile = nxt;
-        if (t + npairs < L.ntiles) nxt = load_tile(L.tiles, t + npairs);  // in flight during this tile
+        const int tn = rd.pop(sh, abort_flag, lim);  // claimed ahead by the producer
+        if (tn < 0) {
+            ok = false;
+            break;
+        }
+        if (tn < L.ntiles) nxt = load_tile(L.tiles, tn);  // in flight during this tile
         const int K = static_cast<int>(tile.kf & kTileMaxK);
         const unsigned fl = tile.kf >> 24;
         const int a_mn = (fl & TILE_A_MN) ? 1 : 0, b_mn = (fl & TILE_B_MN) ? 1 : 0;
@@ -240,14 +328,14 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
         const int fmt = (fl & TILE_BF16) ? 1 : 0;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         const int nk = (K + BK - 1) / BK;
-        if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag)) {
+        if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag, lim)) {
             ok = false;
             break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < nk; ++kb) {
-            if (!mbar_wait(&sh->full[stage], phase, abort_flag)) {
+            if (!mbar_wait(&sh->full[stage], phase, abort_flag, lim)) {
                 ok = false;
                 break;
             }
@@ -280,6 +368,7 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             acc = 0;
             acc_phase ^= 1u;
         }
+        t = tn;
     }
     if (!ok) {
         record_timeout(sh, L.status);
@@ -287,14 +376,15 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             // wait for this thread's MMAs before TMEM is released
             int never = 0;
             umma_commit_pair(&sh->drain, 0x1);
-            if (!mbar_wait(&sh->drain, 0, &never)) atomicOr(&L.status->bits, ST_TIMEOUT);
+            if (!mbar_wait(&sh->drain, 0, &never, lim)) atomicOr(&L.status->bits, ST_TIMEOUT);
         }
     }
 }
 
 __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint32_t tmem_base, int warp, int lane,
-                               uint32_t rank, int pair, int npairs) {
+                               uint32_t rank) {
     volatile int* abort_flag = &sh->abort;
+    const unsigned long long lim = L.wait_ns;
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;  // column half of the tile
     const uint32_t tempty_leader[2] = {map_to_cta(smem_u32(&sh->tempty[0]), 0),
@@ -307,7 +397,20 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     // this lane's 64-byte row of a store box, 16-byte units swizzled (64-byte mode)
     const uint32_t row_off = static_cast<uint32_t>(lane) * 64;
     const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
-    for (int t = pair; t < L.ntiles; t += npairs) {
+    // lane 0 reads the tile-index ring for the warp (one reader per warp)
+    RingReader rd;
+    auto next_tile = [&]() -> int {
+        int v = 0;
+        if (lane == 0) v = rd.pop(sh, abort_flag, lim);
+        return __shfl_sync(0xffffffffu, v, 0);
+    };
+    int t = next_tile();
+    while (t >= 0 && t < L.ntiles) {
+        const int tn = next_tile();  // claimed ahead by the producer
+        if (tn < 0) {
+            if (lane == 0) record_timeout(sh, L.status);
+            break;
+        }
         const TcTile tile = load_tile(L.tiles, t);
         // Local copies: the epilogue stores to global memory, so fields read
         // through a reference into the problem table would be reloaded after
@@ -317,7 +420,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         // the epilogue inputs (C1) come from earlier slots: acquire them too
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
-            if (lane == 0) (void)wait_counter(L.done + tile.mat, tile.need, abort_flag);
+            if (lane == 0) (void)wait_counter(L.done + tile.mat, tile.need, abort_flag, lim);
             __syncwarp();
             seen_mat = tile.mat;
             seen_done = tile.need;
@@ -347,7 +450,10 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             const int bytes = min(BN / 2, PN - cbase) * es;
             for (int o = 0; o < bytes; o += 128) prefetch_l2(p + o);
         }
-        if (!mbar_wait(&sh->tfull[acc], acc_phase, abort_flag)) {
+        // every lane waits; the warp leaves together unless all lanes saw the
+        // accumulator arrive (a lane's wait may end just before the arrival)
+        const bool got = mbar_wait(&sh->tfull[acc], acc_phase, abort_flag, lim);
+        if (!__all_sync(0xffffffffu, got)) {
             if (lane == 0) record_timeout(sh, L.status);
             break;
         }
@@ -433,7 +539,9 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             acc = 0;
             acc_phase ^= 1u;
         }
+        t = tn;
     }
+    if (t < 0 && lane == 0) record_timeout(sh, L.status);
     // the staging boxes must stay valid until every store has read them
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -448,7 +556,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     Shared* sh = reinterpret_cast<Shared*>(store_smem + STORE_BYTES);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_cta_rank();
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -458,6 +565,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sh->tfull[a], 1);
             mbar_init(&sh->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
+        }
+        for (int r = 0; r < SCHED; ++r) {
+            mbar_init(&sh->sfull[r], 1);              // the leader's producer publishes
+            mbar_init(&sh->sempty[r], SCHED_READERS);  // used in the leader only
         }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
@@ -474,12 +585,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem_base = sh->tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) producer(L, tiles_smem, sh, rank, pair, npairs);
+        if (lane == 0) producer(L, tiles_smem, sh, rank);
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base, pair, npairs);
+        if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base);
     } else {
-        epilogue_warps(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank,
-                       pair, npairs);
+        epilogue_warps(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank);
     }
 
     tc_fence_before();

@@ -29,6 +29,11 @@ static_assert(sizeof(TcTile) == 32, "tile records are loaded as two 16-byte vect
 enum { TILE_A_MN = 1, TILE_B_MN = 2, TILE_A_SYM = 4, TILE_B_SYM = 8, TILE_BF16 = 16 };
 constexpr unsigned kTileMaxK = (1u << 24) - 1;
 
+// Tiles are claimed in list order from `ticket` (a global counter, zero at
+// launch): a CTA pair processes the tiles it claims in the order it claimed
+// them.  Every dependency of a tile is on tiles earlier in the list, which
+// are therefore already owned by pairs that are running, whichever pairs of
+// the grid the hardware has made resident.
 struct TcLaunch {
     const TcProblem* problems;
     const TcTile* tiles;
@@ -36,6 +41,8 @@ struct TcLaunch {
     const CUtensorMap* maps;
     const int* bad;       // per-matrix non-finite flags
     unsigned* done;       // per-matrix completion counters (zeroed before the launch), or null
+    unsigned* ticket;     // next unclaimed tile (zeroed before the launch)
+    unsigned long long wait_ns;  // bound of every wait of the launch
     DeviceStatus* status;
 };
 
@@ -55,6 +62,24 @@ struct F32Launch {
 };
 cudaError_t launch_gemm_f32(const F32Launch& L, cudaStream_t stream);
 
+// AdamW lane: one tensor (flat) of the grouped elementwise launch.
+struct AdamTensor {
+    void* p;          // parameter (fp32 or bf16)
+    const void* g;    // gradient (bf16 or fp32)
+    float* m;         // first moment (fp32)
+    float* v;         // second moment (fp32)
+    long long numel;
+    long long chunk_begin;
+    int vec_ok;       // numel % 8 == 0 and every pointer 16-byte aligned (8-element access)
+};
+
+struct AdamLaunch {
+    const AdamTensor* tensors;
+    int ntensors;
+    long long nchunks;
+    int p_dt, g_dt;
+    float decay, beta1, beta2, lr_c1, c2, eps;
+};
 struct MomLaunch {
     const MomMatrix* mats;
     int nmats;
@@ -74,8 +99,11 @@ struct MomLaunch {
     int* bad;           // per matrix non-finite flag
     DeviceStatus* status;
     int mat_index_base; // index of mats[0] in the caller's numbering (status reporting)
-    unsigned* done;     // GEMM completion counters to zero for the next chain launch (or null)
+    unsigned* done;     // GEMM completion counters and tile tickets to zero for the GEMM launches that follow
     int ndone;
+    // hybrid step: the AdamW lane's chunks follow the nchunks Muon chunks in
+    // the same grid (adam.ntensors == 0: none); its gradients share in_dt
+    AdamLaunch adam;
 };
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream);
 
@@ -91,24 +119,6 @@ struct ScaleLaunch {
 };
 cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream);
 
-// AdamW lane: one tensor (flat) of the grouped elementwise launch.
-struct AdamTensor {
-    void* p;          // parameter (fp32 or bf16)
-    const void* g;    // gradient (bf16 or fp32)
-    float* m;         // first moment (fp32)
-    float* v;         // second moment (fp32)
-    long long numel;
-    long long chunk_begin;
-    int vec_ok;       // numel % 8 == 0 and every pointer 16-byte aligned (8-element access)
-};
-
-struct AdamLaunch {
-    const AdamTensor* tensors;
-    int ntensors;
-    long long nchunks;
-    int p_dt, g_dt;
-    float decay, beta1, beta2, lr_c1, c2, eps;
-};
 cudaError_t launch_adamw(const AdamLaunch& L, cudaStream_t stream);
 
 // The stream bound by muon_set_stream, and the message muon_last_error returns.

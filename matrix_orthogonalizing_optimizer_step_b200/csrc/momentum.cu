@@ -18,6 +18,7 @@
 // flags non-finite norms, and resets the ticket for the next launch.
 #include <cuda_bf16.h>
 
+#include "adamw.cuh"
 #include "epilogue.cuh"
 #include "launch.h"
 
@@ -86,7 +87,15 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     __shared__ double red_d[kThreads / 32];
     __shared__ int is_last;
     const long long chunk = blockIdx.x;
-    if (chunk == 0 && L.done)  // the chained GEMM that follows counts tile completions from zero
+    if (chunk >= L.nchunks) {
+        // hybrid step: the AdamW lane's chunks follow the Muon chunks
+        if (L.adam.p_dt == DT_F32)
+            adamw_chunk<true, G_F32>(L.adam, chunk - L.nchunks);
+        else
+            adamw_chunk<false, G_F32>(L.adam, chunk - L.nchunks);
+        return;
+    }
+    if (chunk == 0 && L.done)  // the GEMM launches that follow count completions and tickets from zero
         for (int i = threadIdx.x; i < L.ndone; i += kThreads) L.done[i] = 0u;
     const int mi = find_matrix(L.nmats, chunk, L.mats);
     const MomMatrix Mx = L.mats[mi];  // local copy: no reloads after global stores
@@ -160,10 +169,13 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     const double total = block_sum<double>(acc, red_d);
     if (threadIdx.x == 0) {
         const bool finite = isfinite(total);
-        const double s = 1.0 / (sqrt(total) + L.eps);
-        L.scale[4 * mi] = finite ? static_cast<float>(s) : 0.f;
-        L.scale[4 * mi + 1] = finite ? static_cast<float>(s * s) : 0.f;
-        L.scale[4 * mi + 2] = finite ? static_cast<float>(-static_cast<double>(L.lr) * s) : 0.f;
+        // a zero matrix with eps = 0 has no scale: s = 0 (its outputs are 0
+        // and its parameter does not move), not 1/0
+        const double denom = sqrt(total) + L.eps;
+        const double s = (finite && denom > 0.0) ? 1.0 / denom : 0.0;
+        L.scale[4 * mi] = static_cast<float>(s);
+        L.scale[4 * mi + 1] = static_cast<float>(s * s);
+        L.scale[4 * mi + 2] = static_cast<float>(-static_cast<double>(L.lr) * s);
         L.scale[4 * mi + 3] = finite ? -L.lr : 0.f;
         L.bad[mi] = finite ? 0 : 1;
         if (!finite) {
@@ -223,7 +235,8 @@ static cudaError_t launch_step(const MomLaunch& L, dim3 grid, bool gf, cudaStrea
 
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream) {
     if (L.nchunks <= 0) return cudaSuccess;
-    const dim3 grid(static_cast<unsigned>(L.nchunks));
+    if (L.adam.ntensors > 0 && (!L.has_momentum || L.adam.g_dt != L.in_dt)) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(L.nchunks + (L.adam.ntensors > 0 ? L.adam.nchunks : 0)));
     const bool gf = L.in_dt == DT_F32, uf = L.u_dt == DT_F32;
     if (!L.has_momentum) {
         if (gf && uf)

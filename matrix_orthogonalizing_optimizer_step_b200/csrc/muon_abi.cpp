@@ -3,6 +3,7 @@
 // No exception crosses this boundary; every entry point returns a status.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -35,8 +36,23 @@ struct DeviceState {
     void* adam_table = nullptr;  // AdamW tensor table
     size_t adam_cap = 0;
     std::vector<AdamTensor> adam_last;  // contents of adam_table
+    // The workspace (plan tables, intermediates, AdamW table) is reused by
+    // every call.  ws_event marks the end of its last use, on ws_stream; a
+    // call on another stream first makes its stream wait for that event, so
+    // its table uploads and kernels cannot overlap the previous call's.
+    cudaEvent_t ws_event = nullptr;
+    cudaStream_t ws_stream = nullptr;
+    bool ws_used = false;
 };
 std::deque<DeviceState> g_devs;  // deque: references stay valid on growth
+
+// Per-shape Newton-Schulz schedules of muon_step, keyed by the short and the
+// long side of the matrix.
+struct ShapeSchedule {
+    int n, m, steps;
+    std::vector<float> coeffs;
+};
+std::vector<ShapeSchedule> g_shape_scheds;
 
 int fail(int code, const std::string& msg) {
     g_err = msg;
@@ -112,6 +128,11 @@ int device_state(DeviceState** out) {
     }
     const DeviceStatus init{0, 0x7fffffff};
     cudaMemcpy(d.status, &init, sizeof(init), cudaMemcpyHostToDevice);
+    if (cudaEventCreateWithFlags(&d.ws_event, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(d.status);
+        return fail(MUON_ERR_CUDA, "event creation failed");
+    }
     d.plan.reset(new Plan());
     g_devs.push_back(std::move(d));
     *out = &g_devs.back();
@@ -187,9 +208,38 @@ struct Profiler : ProfileSink {
 };
 Profiler g_prof;
 
-int run_plan(DeviceState* ds, const PlanRequest& rq) {
+// Order this call's use of the workspace after its last use on another stream.
+int ws_acquire(DeviceState* ds) {
+    if (ds->ws_used && ds->ws_stream != g_stream) {
+        const cudaError_t e = cudaStreamWaitEvent(g_stream, ds->ws_event, 0);
+        if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("stream wait failed: ") + cudaGetErrorString(e));
+    }
+    return MUON_OK;
+}
+
+// Mark the end of this call's use of the workspace on the bound stream.
+int ws_release(DeviceState* ds) {
+    const cudaError_t e = cudaEventRecord(ds->ws_event, g_stream);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("event record failed: ") + cudaGetErrorString(e));
+    ds->ws_stream = g_stream;
+    ds->ws_used = true;
+    return MUON_OK;
+}
+
+// An AdamW lane, checked and ready to launch.
+struct AdamArgs {
+    std::vector<AdamTensor> t;
+    AdamLaunch L{};
+    double bytes = 0;  // algorithmic HBM bytes
+};
+
+// Run the plan of rq (built or reused).  With `adam`, the AdamW lane's chunks
+// are appended to the grid of the plan's momentum launch.
+int run_plan(DeviceState* ds, const PlanRequest& rq, const AdamArgs* adam) {
     std::string err;
     Plan& plan = *ds->plan;
+    int wst = ws_acquire(ds);
+    if (wst != MUON_OK) return wst;
     if (!plan.same_shape_key(rq)) {
         // tables of the previous plan may still be read by queued kernels
         cudaError_t e = cudaStreamSynchronize(g_stream);
@@ -201,10 +251,152 @@ int run_plan(DeviceState* ds, const PlanRequest& rq) {
         }
     }
     plan.set_scalars(rq.mu, rq.nesterov, rq.lr, rq.clip);
+    plan.set_adamw(adam ? &adam->L : nullptr, adam ? adam->bytes : 0.0);
     long long launched = 0;
     const int st = plan.run(g_stream, g_prof.on ? &g_prof : nullptr, &launched, err);
     g_launches += launched;
+    wst = ws_release(ds);
     if (st != MUON_OK) return fail(st, err);
+    return wst;
+}
+
+// ---- argument checks shared by the step entry points (host only) ----------------
+
+// Validate the Muon lane of a step and describe it as a plan request (no device work).
+int step_request(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
+                 float lr, const int* shape_list, int count, PlanRequest& rq) {
+    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
+    if (!params || !grads || !momentum || !shape_list)
+        return fail(MUON_ERR_INVALID_ARG, "params, grads, momentum and shape_list must not be NULL");
+    if (!std::isfinite(mu) || !std::isfinite(lr)) return fail(MUON_ERR_INVALID_ARG, "mu and lr must be finite");
+    for (int i = 0; i < count; ++i) {
+        const int r = shape_list[2 * i], c = shape_list[2 * i + 1];
+        if (r < 1 || c < 1) return fail(MUON_ERR_INVALID_ARG, "shape_list entries must be >= 1");
+        if (!params[i] || !grads[i] || !momentum[i])
+            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/momentum");
+        rq.rows.push_back(r);
+        rq.cols.push_back(c);
+        rq.in.push_back(grads[i]);
+        rq.mom.push_back(momentum[i]);
+        rq.out.push_back(params[i]);
+    }
+    rq.in_dt = g_cfg.grad_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
+    rq.mom_dt = g_cfg.momentum_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
+    rq.out_dt = g_cfg.param_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
+    rq.is_step = true;
+    rq.fp32_path = false;
+    rq.form = g_cfg.mode;
+    rq.steps = g_cfg.steps;
+    rq.coeffs.assign(g_cfg.coeffs, g_cfg.coeffs + 3 * g_cfg.steps);
+    rq.restart_mask = g_cfg.restart_mask;
+    rq.eps = g_cfg.eps;
+    rq.mu = mu;
+    rq.nesterov = nesterov ? 1 : 0;
+    rq.lr = lr;
+    rq.clip = 0.5f * g_cfg.soft_threshold;
+    if (!g_shape_scheds.empty()) {
+        // each matrix takes the schedule registered for its shape, if any
+        std::vector<int> used(g_shape_scheds.size(), -1);
+        rq.sched.assign(count, -1);
+        for (int i = 0; i < count; ++i) {
+            const int n = std::min(rq.rows[i], rq.cols[i]), m = std::max(rq.rows[i], rq.cols[i]);
+            for (size_t e = 0; e < g_shape_scheds.size(); ++e) {
+                if (g_shape_scheds[e].n != n || g_shape_scheds[e].m != m) continue;
+                if (used[e] < 0) {
+                    used[e] = static_cast<int>(rq.scheds.size());
+                    PlanRequest::Schedule sc;
+                    sc.steps = g_shape_scheds[e].steps;
+                    sc.coeffs = g_shape_scheds[e].coeffs;
+                    rq.scheds.push_back(sc);
+                }
+                rq.sched[i] = used[e];
+                break;
+            }
+        }
+    }
+    return MUON_OK;
+}
+
+// Validate an AdamW lane and build its launch description (no device work).
+int adamw_prepare(void* const* params, const void* const* grads, void* const* exp_avg, void* const* exp_avg_sq,
+                  const long long* numels, int count, float lr, float beta1, float beta2, float eps,
+                  float weight_decay, int step, AdamArgs& out) {
+    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
+    if (!params || !grads || !exp_avg || !exp_avg_sq || !numels)
+        return fail(MUON_ERR_INVALID_ARG, "params, grads, exp_avg, exp_avg_sq and numels must not be NULL");
+    if (step < 1) return fail(MUON_ERR_INVALID_ARG, "step must be >= 1");
+    if (!std::isfinite(lr) || !std::isfinite(weight_decay) || !(eps >= 0.f) || !std::isfinite(eps) ||
+        !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
+        return fail(MUON_ERR_INVALID_ARG, "lr, weight_decay, eps finite; 0 <= beta1, beta2 < 1");
+    std::vector<AdamTensor>& t = out.t;
+    t.assign(count, AdamTensor{});
+    long long chunks = 0;
+    const bool pf32 = g_cfg.param_dtype == MUON_DTYPE_F32;
+    const bool gf32 = g_cfg.grad_dtype == MUON_DTYPE_F32;
+    double elems = 0;
+    for (int i = 0; i < count; ++i) {
+        if (numels[i] < 1) return fail(MUON_ERR_INVALID_ARG, "numels entries must be >= 1");
+        if (!params[i] || !grads[i] || !exp_avg[i] || !exp_avg_sq[i])
+            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/exp_avg/exp_avg_sq");
+        t[i].p = params[i];
+        t[i].g = grads[i];
+        t[i].m = static_cast<float*>(exp_avg[i]);
+        t[i].v = static_cast<float*>(exp_avg_sq[i]);
+        t[i].numel = numels[i];
+        t[i].chunk_begin = chunks;
+        auto al = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+        t[i].vec_ok = numels[i] % 8 == 0 && al(params[i], 16) && al(grads[i], 16) && al(exp_avg[i], 16) &&
+                      al(exp_avg_sq[i], 16);
+        chunks += (numels[i] + kMomChunk - 1) / kMomChunk;
+        elems += static_cast<double>(numels[i]);
+    }
+    AdamLaunch& L = out.L;
+    L.tensors = nullptr;  // set by adamw_upload
+    L.ntensors = count;
+    L.nchunks = chunks;
+    L.p_dt = pf32 ? DT_F32 : DT_BF16;
+    L.g_dt = gf32 ? DT_F32 : DT_BF16;
+    L.decay = static_cast<float>(1.0 - static_cast<double>(lr) * weight_decay);
+    L.beta1 = beta1;
+    L.beta2 = beta2;
+    L.lr_c1 = static_cast<float>(static_cast<double>(lr) / (1.0 - std::pow(static_cast<double>(beta1), step)));
+    L.c2 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(beta2), step)));
+    L.eps = eps;
+    out.bytes = elems * ((pf32 ? 8.0 : 4.0) + (gf32 ? 4.0 : 2.0) + 16.0);
+    return MUON_OK;
+}
+
+// Upload the AdamW tensor table into the library's buffer (after ws_acquire).
+int adamw_upload(DeviceState* ds, AdamArgs& aa) {
+    // the tensor table lives in a small device buffer owned by the library;
+    // a previous launch on the bound stream (or, through ws_acquire, on the
+    // stream of the previous call) has read it before this upload runs
+    std::vector<AdamTensor>& last = ds->adam_last;
+    const std::vector<AdamTensor>& t = aa.t;
+    const size_t bytes = sizeof(AdamTensor) * t.size();
+    if (ds->adam_cap < bytes) {
+        if (ds->adam_table) {
+            cudaStreamSynchronize(g_stream);
+            cudaFree(ds->adam_table);
+        }
+        ds->adam_table = nullptr;
+        ds->adam_cap = 0;
+        const char* fault = std::getenv("MUON_FAULT");
+        if (fault && !std::strcmp(fault, "alloc"))  // injected failure (see the planner's MUON_FAULT)
+            return fail(MUON_ERR_NO_MEMORY, "AdamW table allocation failed (injected: MUON_FAULT=alloc)");
+        if (cudaMalloc(&ds->adam_table, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return fail(MUON_ERR_NO_MEMORY, "AdamW table allocation failed");
+        }
+        ds->adam_cap = bytes;
+        last.clear();
+    }
+    if (last.size() != t.size() || std::memcmp(last.data(), t.data(), bytes) != 0) {
+        cudaError_t e = cudaMemcpyAsync(ds->adam_table, t.data(), bytes, cudaMemcpyHostToDevice, g_stream);
+        if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table upload failed: ") + cudaGetErrorString(e));
+        last = t;
+    }
+    aa.L.tensors = static_cast<const AdamTensor*>(ds->adam_table);
     return MUON_OK;
 }
 
@@ -258,8 +450,24 @@ const char* muon_last_error(void) { return g_err.c_str(); }
 
 int muon_release_workspace(void) {
     cudaStreamSynchronize(g_stream);
-    for (DeviceState& d : g_devs)
+    int cur = -1;
+    cudaGetDevice(&cur);
+    for (DeviceState& d : g_devs) {
+        if (d.ws_used) {
+            cudaSetDevice(d.device);
+            cudaEventSynchronize(d.ws_event);  // the last use, on whichever stream
+            d.ws_used = false;
+        }
         if (d.plan) d.plan->release();
+        if (d.adam_table) {
+            cudaSetDevice(d.device);
+            cudaFree(d.adam_table);
+            d.adam_table = nullptr;
+            d.adam_cap = 0;
+            d.adam_last.clear();
+        }
+    }
+    if (cur >= 0) cudaSetDevice(cur);
     return MUON_OK;
 }
 
@@ -318,125 +526,107 @@ int muon_orthogonalize(int batch, int m, int n, void* X, const float* coeffs, in
     rq.restart_mask = g_cfg.restart_mask;
     rq.eps = g_cfg.eps;
     rq.device = ds->device;
-    return run_plan(ds, rq);
+    return run_plan(ds, rq, nullptr);
 }
 
 int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov, float lr,
               const int* shape_list, int count) {
     ensure_cfg();
-    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
-    if (!params || !grads || !momentum || !shape_list)
-        return fail(MUON_ERR_INVALID_ARG, "params, grads, momentum and shape_list must not be NULL");
-    if (!std::isfinite(mu) || !std::isfinite(lr)) return fail(MUON_ERR_INVALID_ARG, "mu and lr must be finite");
     PlanRequest rq;
-    for (int i = 0; i < count; ++i) {
-        const int r = shape_list[2 * i], c = shape_list[2 * i + 1];
-        if (r < 1 || c < 1) return fail(MUON_ERR_INVALID_ARG, "shape_list entries must be >= 1");
-        if (!params[i] || !grads[i] || !momentum[i])
-            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/momentum");
-        rq.rows.push_back(r);
-        rq.cols.push_back(c);
-        rq.in.push_back(grads[i]);
-        rq.mom.push_back(momentum[i]);
-        rq.out.push_back(params[i]);
-    }
-    DeviceState* ds = nullptr;
-    int st = check_device(&ds, true);
+    int st = step_request(params, grads, momentum, mu, nesterov, lr, shape_list, count, rq);
     if (st != MUON_OK) return st;
-    rq.in_dt = g_cfg.grad_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
-    rq.mom_dt = g_cfg.momentum_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
-    rq.out_dt = g_cfg.param_dtype == MUON_DTYPE_F32 ? DT_F32 : DT_BF16;
-    rq.is_step = true;
-    rq.fp32_path = false;
-    rq.form = g_cfg.mode;
-    rq.steps = g_cfg.steps;
-    rq.coeffs.assign(g_cfg.coeffs, g_cfg.coeffs + 3 * g_cfg.steps);
-    rq.restart_mask = g_cfg.restart_mask;
-    rq.eps = g_cfg.eps;
-    rq.mu = mu;
-    rq.nesterov = nesterov ? 1 : 0;
-    rq.lr = lr;
-    rq.clip = 0.5f * g_cfg.soft_threshold;
+    DeviceState* ds = nullptr;
+    st = check_device(&ds, true);
+    if (st != MUON_OK) return st;
     rq.device = ds->device;
-    return run_plan(ds, rq);
+    return run_plan(ds, rq, nullptr);
+}
+
+int muon_hybrid_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
+                     float lr, const int* shape_list, int count, const muon_adamw_lane* adamw) {
+    ensure_cfg();
+    if (!adamw) return fail(MUON_ERR_INVALID_ARG, "adamw is NULL");
+    PlanRequest rq;
+    int st = step_request(params, grads, momentum, mu, nesterov, lr, shape_list, count, rq);
+    if (st != MUON_OK) return st;
+    AdamArgs aa;
+    st = adamw_prepare(adamw->params, adamw->grads, adamw->exp_avg, adamw->exp_avg_sq, adamw->numels, adamw->count,
+                       adamw->lr, adamw->beta1, adamw->beta2, adamw->eps, adamw->weight_decay, adamw->step, aa);
+    if (st != MUON_OK) return st;
+    DeviceState* ds = nullptr;
+    st = check_device(&ds, true);
+    if (st != MUON_OK) return st;
+    rq.device = ds->device;
+    st = ws_acquire(ds);
+    if (st != MUON_OK) return st;
+    st = adamw_upload(ds, aa);
+    if (st != MUON_OK) return st;
+    return run_plan(ds, rq, &aa);
+}
+
+int muon_set_shape_coeffs(int rows, int cols, const float* coeffs, int steps) {
+    if (rows < 1 || cols < 1) return fail(MUON_ERR_INVALID_ARG, "rows and cols must be >= 1");
+    if (steps < 0 || steps > MUON_MAX_STEPS) return fail(MUON_ERR_INVALID_ARG, "steps out of range");
+    if (steps > 0 && !coeffs) return fail(MUON_ERR_INVALID_ARG, "coeffs is NULL");
+    for (int i = 0; i < 3 * steps; ++i)
+        if (!std::isfinite(coeffs[i])) return fail(MUON_ERR_INVALID_ARG, "coeffs must be finite");
+    const int n = std::min(rows, cols), m = std::max(rows, cols);
+    for (ShapeSchedule& e : g_shape_scheds)
+        if (e.n == n && e.m == m) {
+            e.steps = steps;
+            e.coeffs.assign(coeffs, coeffs + 3 * steps);
+            return MUON_OK;
+        }
+    if (static_cast<int>(g_shape_scheds.size()) >= MUON_MAX_SHAPE_SCHEDULES)
+        return fail(MUON_ERR_INVALID_ARG, "more than MUON_MAX_SHAPE_SCHEDULES shapes registered");
+    ShapeSchedule e;
+    e.n = n;
+    e.m = m;
+    e.steps = steps;
+    e.coeffs.assign(coeffs, coeffs + 3 * steps);
+    g_shape_scheds.push_back(e);
+    return MUON_OK;
+}
+
+int muon_get_shape_coeffs(int rows, int cols, float* coeffs, int* steps) {
+    if (rows < 1 || cols < 1 || !steps) return fail(MUON_ERR_INVALID_ARG, "rows, cols >= 1 and steps not NULL");
+    const int n = std::min(rows, cols), m = std::max(rows, cols);
+    for (const ShapeSchedule& e : g_shape_scheds)
+        if (e.n == n && e.m == m) {
+            *steps = e.steps;
+            if (coeffs) std::copy(e.coeffs.begin(), e.coeffs.end(), coeffs);
+            return MUON_OK;
+        }
+    *steps = -1;
+    return MUON_OK;
+}
+
+int muon_clear_shape_coeffs(void) {
+    g_shape_scheds.clear();
+    return MUON_OK;
 }
 
 int muon_adamw_step(void* const* params, const void* const* grads, void* const* exp_avg, void* const* exp_avg_sq,
                     const long long* numels, int count, float lr, float beta1, float beta2, float eps,
                     float weight_decay, int step) {
     ensure_cfg();
-    if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
-    if (!params || !grads || !exp_avg || !exp_avg_sq || !numels)
-        return fail(MUON_ERR_INVALID_ARG, "params, grads, exp_avg, exp_avg_sq and numels must not be NULL");
-    if (step < 1) return fail(MUON_ERR_INVALID_ARG, "step must be >= 1");
-    if (!std::isfinite(lr) || !std::isfinite(weight_decay) || !(eps >= 0.f) || !std::isfinite(eps) ||
-        !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f))
-        return fail(MUON_ERR_INVALID_ARG, "lr, weight_decay, eps finite; 0 <= beta1, beta2 < 1");
-    std::vector<AdamTensor> t(count);
-    long long chunks = 0;
-    const bool pf32 = g_cfg.param_dtype == MUON_DTYPE_F32;
-    const bool gf32 = g_cfg.grad_dtype == MUON_DTYPE_F32;
-    for (int i = 0; i < count; ++i) {
-        if (numels[i] < 1) return fail(MUON_ERR_INVALID_ARG, "numels entries must be >= 1");
-        if (!params[i] || !grads[i] || !exp_avg[i] || !exp_avg_sq[i])
-            return fail(MUON_ERR_INVALID_ARG, "null pointer in params/grads/exp_avg/exp_avg_sq");
-        t[i].p = params[i];
-        t[i].g = grads[i];
-        t[i].m = static_cast<float*>(exp_avg[i]);
-        t[i].v = static_cast<float*>(exp_avg_sq[i]);
-        t[i].numel = numels[i];
-        t[i].chunk_begin = chunks;
-        auto al = [](const void* p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
-        t[i].vec_ok = numels[i] % 8 == 0 && al(params[i], 16) && al(grads[i], 16) && al(exp_avg[i], 16) &&
-                      al(exp_avg_sq[i], 16);
-        chunks += (numels[i] + kMomChunk - 1) / kMomChunk;
-    }
-    DeviceState* ds = nullptr;
-    int st = check_device(&ds, false);
+    AdamArgs aa;
+    int st = adamw_prepare(params, grads, exp_avg, exp_avg_sq, numels, count, lr, beta1, beta2, eps, weight_decay,
+                           step, aa);
     if (st != MUON_OK) return st;
-    // the tensor table lives in a small device buffer owned by the library;
-    // a previous launch on the bound stream has read it before this upload runs
-    std::vector<AdamTensor>& last = ds->adam_last;
-    const size_t bytes = sizeof(AdamTensor) * t.size();
-    if (ds->adam_cap < bytes) {
-        if (ds->adam_table) {
-            cudaStreamSynchronize(g_stream);
-            cudaFree(ds->adam_table);
-        }
-        ds->adam_table = nullptr;
-        ds->adam_cap = 0;
-        if (cudaMalloc(&ds->adam_table, bytes) != cudaSuccess) {
-            cudaGetLastError();
-            return fail(MUON_ERR_NO_MEMORY, "AdamW table allocation failed");
-        }
-        ds->adam_cap = bytes;
-        last.clear();
-    }
-    if (last.size() != t.size() || std::memcmp(last.data(), t.data(), bytes) != 0) {
-        cudaError_t e = cudaMemcpyAsync(ds->adam_table, t.data(), bytes, cudaMemcpyHostToDevice, g_stream);
-        if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table upload failed: ") + cudaGetErrorString(e));
-        last = t;
-    }
-    AdamLaunch L;
-    L.tensors = static_cast<const AdamTensor*>(ds->adam_table);
-    L.ntensors = count;
-    L.nchunks = chunks;
-    L.p_dt = pf32 ? DT_F32 : DT_BF16;
-    L.g_dt = gf32 ? DT_F32 : DT_BF16;
-    L.decay = static_cast<float>(1.0 - static_cast<double>(lr) * weight_decay);
-    L.beta1 = beta1;
-    L.beta2 = beta2;
-    L.lr_c1 = static_cast<float>(static_cast<double>(lr) / (1.0 - std::pow(static_cast<double>(beta1), step)));
-    L.c2 = static_cast<float>(1.0 / (1.0 - std::pow(static_cast<double>(beta2), step)));
-    L.eps = eps;
+    DeviceState* ds = nullptr;
+    st = check_device(&ds, false);
+    if (st != MUON_OK) return st;
+    st = ws_acquire(ds);
+    if (st != MUON_OK) return st;
+    st = adamw_upload(ds, aa);
+    if (st != MUON_OK) return st;
     if (g_prof.on) g_prof.before(g_stream);
-    cudaError_t e = launch_adamw(L, g_stream);
+    cudaError_t e = launch_adamw(aa.L, g_stream);
     if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(e));
     ++g_launches;
-    double elems = 0;
-    for (const AdamTensor& x : t) elems += static_cast<double>(x.numel);
-    if (g_prof.on) g_prof.after(g_stream, 4, 0.0, elems * ((pf32 ? 8.0 : 4.0) + (gf32 ? 4.0 : 2.0) + 16.0));
-    return MUON_OK;
+    if (g_prof.on) g_prof.after(g_stream, 4, 0.0, aa.bytes);
+    return ws_release(ds);
 }
 
 int muon_profile_enable(int on) {

@@ -28,7 +28,7 @@ constexpr int kMaxDevices = 64;
 struct NoAllocScratch {
     float partials[MUON_NOALLOC_MAX_CHUNKS];  // one per 8192-element chunk
     int counters[MUON_NOALLOC_MAX_MATRICES];  // ticket per matrix, zero between calls
-    float scale[MUON_NOALLOC_MAX_MATRICES];   // 1 / (||X_i|| + eps), 0 if not finite
+    float scale[MUON_NOALLOC_MAX_MATRICES];   // 1 / (||X_i|| + eps); NaN if the norm is not finite
 };
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoAllocScratch)];
@@ -87,7 +87,11 @@ __global__ void __launch_bounds__(kThreads) noalloc_norm_kernel(const void* X, i
         acc += static_cast<double>(__ldcg(&S->partials[static_cast<long long>(mat) * chunks_per_mat + i]));
     const double total = block_sum<double>(acc, red_d);
     if (threadIdx.x == 0) {
-        S->scale[mat] = isfinite(total) ? static_cast<float>(1.0 / (sqrt(total) + eps)) : 0.f;
+        // non-finite norm: NaN marks the matrix as left untouched; a zero
+        // matrix with eps = 0 gets s = 0 (its output is 0), not 1/0
+        const double denom = sqrt(total) + eps;
+        S->scale[mat] = !isfinite(total) ? __int_as_float(0x7fc00000)
+                                         : (denom > 0.0 ? static_cast<float>(1.0 / denom) : 0.f);
         S->counters[mat] = 0;
     }
 }
@@ -98,7 +102,7 @@ __global__ void __launch_bounds__(kThreads) noalloc_scale_kernel(const void* X, 
     const long long chunk = blockIdx.x;
     const int mat = static_cast<int>(chunk / chunks_per_mat);
     const float s = S->scale[mat];
-    if (s == 0.f) return;
+    if (s != s) return;  // non-finite norm: Y untouched
     const long long e0 = (chunk % chunks_per_mat) * kMomChunk;
     const long long base = static_cast<long long>(mat) * numel;
     for (int i = threadIdx.x; i < kMomChunk; i += kThreads) {

@@ -50,6 +50,8 @@ struct Group {
     int n = 0, m = 0;
     bool trans = false;
     int form = FORM_STANDARD;
+    int steps = 0;              // Newton-Schulz steps of this group's schedule
+    std::vector<float> coeffs;  // (a, b, c) of step k at [3k .. 3k+2]
     std::vector<int> mats;
     long long rows_w = 0, cols_w = 0;  // X buffers in the caller's layout
     long long ldx = 0, ldn = 0;
@@ -61,6 +63,32 @@ struct Group {
 };
 
 long long round_up(long long v, long long a) { return (v + a - 1) / a * a; }
+
+// Host-side fault injection for the failure-path tests (MUON_FAULT):
+//   alloc    the workspace allocation of a plan build fails (MUON_ERR_NO_MEMORY)
+//   launch   the first kernel launch of a call fails (MUON_ERR_CUDA)
+//   timeout  the first tile of a chained launch waits on a completion count
+//            that is never reached, so its bounded wait runs out
+//            (MUON_ERR_TIMEOUT through the device status word)
+// No fault is injected on the device: the kernels only see a dependency
+// count that no tile will satisfy, and give up after their wait limit.
+enum Fault { FAULT_NONE = 0, FAULT_ALLOC, FAULT_LAUNCH, FAULT_TIMEOUT };
+int fault_mode() {
+    const char* f = std::getenv("MUON_FAULT");
+    if (!f) return FAULT_NONE;
+    if (!std::strcmp(f, "alloc")) return FAULT_ALLOC;
+    if (!std::strcmp(f, "launch")) return FAULT_LAUNCH;
+    if (!std::strcmp(f, "timeout")) return FAULT_TIMEOUT;
+    return FAULT_NONE;
+}
+
+// Bound of every device-side wait (MUON_WAIT_LIMIT_MS, 1 ms .. 10 s; default 1 s).
+unsigned long long wait_limit_ns() {
+    const char* v = std::getenv("MUON_WAIT_LIMIT_MS");
+    long long ms = v ? std::atoll(v) : 1000;
+    ms = std::max(1LL, std::min(ms, 10000LL));
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+}
 
 bool restart_at(unsigned mask, int k) { return k > 0 && k < 32 && ((mask >> k) & 1u); }
 
@@ -77,12 +105,12 @@ void make_final(OpDesc& op, const PlanRequest& rq) {
 }
 
 void chain_standard(Group& g, const PlanRequest& rq) {
-    const int T = rq.steps;
+    const int T = g.steps;
     int xcur = X0;
     const int xring[2] = {X1, X2};
     int ring = 0;
     for (int k = 0; k < T; ++k) {
-        const float a = rq.coeffs[3 * k], b = rq.coeffs[3 * k + 1], c = rq.coeffs[3 * k + 2];
+        const float a = g.coeffs[3 * k], b = g.coeffs[3 * k + 1], c = g.coeffs[3 * k + 2];
         OpDesc syrk;
         syrk.kind = OP_SYRK;
         syrk.a = syrk.b = xcur;
@@ -119,7 +147,7 @@ void chain_standard(Group& g, const PlanRequest& rq) {
 }
 
 void chain_gram(Group& g, const PlanRequest& rq) {
-    const int T = rq.steps;
+    const int T = g.steps;
     int xcur = X0;
     bool x_scaled = false;  // X0 still carries the factor s
     const int xring[2] = {X1, X2};
@@ -135,7 +163,7 @@ void chain_gram(Group& g, const PlanRequest& rq) {
     }
     int qsrc = -1;  // buffer holding Q, -1 = identity (segment start)
     for (int k = 0; k < T; ++k) {
-        const float a = rq.coeffs[3 * k], b = rq.coeffs[3 * k + 1], c = rq.coeffs[3 * k + 2];
+        const float a = g.coeffs[3 * k], b = g.coeffs[3 * k + 1], c = g.coeffs[3 * k + 2];
         if (restart_at(rq.restart_mask, k)) {
             // X <- Q X, R <- X X^T, Q <- I
             OpDesc app;
@@ -327,11 +355,22 @@ static std::vector<long long> make_key(const PlanRequest& rq) {
     k.push_back(rq.in_dt);
     k.push_back(rq.mom_dt);
     k.push_back(rq.out_dt);
-    for (float c : rq.coeffs) {
-        int bits;
-        std::memcpy(&bits, &c, 4);
-        k.push_back(bits);
+    auto push_coeffs = [&](const std::vector<float>& cs) {
+        for (float c : cs) {
+            int bits;
+            std::memcpy(&bits, &c, 4);
+            k.push_back(bits);
+        }
+    };
+    push_coeffs(rq.coeffs);
+    k.push_back(static_cast<long long>(rq.scheds.size()));
+    for (const PlanRequest::Schedule& sc : rq.scheds) {
+        k.push_back(sc.steps);
+        push_coeffs(sc.coeffs);
     }
+    for (int si : rq.sched) k.push_back(si);
+    k.push_back(fault_mode());
+    k.push_back(static_cast<long long>(wait_limit_ns()));
     for (size_t i = 0; i < rq.rows.size(); ++i) {
         k.push_back(rq.rows[i]);
         k.push_back(rq.cols[i]);
@@ -357,6 +396,18 @@ void Plan::set_scalars(float mu, int nesterov, float lr, float clip) {
     }
 }
 
+void Plan::set_adamw(const AdamLaunch* adam, double bytes) {
+    for (LaunchRec& l : launches)
+        if (l.kind == LaunchRec::MOM) {
+            if (adam) {
+                l.mom.adam = *adam;
+            } else {
+                std::memset(&l.mom.adam, 0, sizeof(l.mom.adam));
+            }
+            l.extra_bytes = adam ? bytes : 0.0;
+        }
+}
+
 void Plan::release() {
     if (arena_) cudaFree(arena_);
     arena_ = nullptr;
@@ -376,14 +427,16 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
 
     // ---- groups ----------------------------------------------------------------
     std::vector<Group> groups;
-    std::map<std::tuple<int, int, int, int>, int> gindex;
+    std::map<std::tuple<int, int, int, int, int>, int> gindex;  // (n, m, trans, form, schedule)
     std::vector<int> mat_group(nm), mat_z(nm);
     for (int i = 0; i < nm; ++i) {
         const int r = rq.rows[i], c = rq.cols[i];
         const bool trans = r > c;
         const int n = trans ? c : r, m = trans ? r : c;
-        const int form = rq.steps > 0 ? resolve_form(n, m, rq.steps, rq.form, rq.restart_mask) : FORM_STANDARD;
-        auto key = std::make_tuple(n, m, static_cast<int>(trans), form);
+        const int si = rq.sched.empty() ? -1 : rq.sched[i];
+        const int steps = si < 0 ? rq.steps : rq.scheds[si].steps;
+        const int form = steps > 0 ? resolve_form(n, m, steps, rq.form, rq.restart_mask) : FORM_STANDARD;
+        auto key = std::make_tuple(n, m, static_cast<int>(trans), form, si);
         auto it = gindex.find(key);
         int gi;
         if (it == gindex.end()) {
@@ -394,6 +447,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
             g.m = m;
             g.trans = trans;
             g.form = form;
+            g.steps = steps;
+            g.coeffs = si < 0 ? rq.coeffs : rq.scheds[si].coeffs;
             g.rows_w = r;
             g.cols_w = c;
             g.ldx = round_up(c, 8);
@@ -414,7 +469,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         }
     }
     for (Group& g : groups) {
-        if (rq.steps > 0) {
+        if (g.steps > 0) {
             if (g.form == FORM_GRAM)
                 chain_gram(g, rq);
             else
@@ -461,7 +516,14 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     const size_t off_counters = take(sizeof(int) * nm);
     const size_t off_scale = take(sizeof(float) * 4 * nm);
     const size_t off_bad = take(sizeof(int) * nm);
-    const size_t off_done = take(sizeof(unsigned) * nm);
+    // per-matrix completion counters, then one tile ticket per GEMM launch
+    // (at most one per chain slot), all zeroed by the momentum kernel
+    const size_t nticket_max = f32 ? 0 : std::max<size_t>(1, [&] {
+        size_t n = 0;
+        for (const Group& g : groups) n = std::max(n, g.slots.size());
+        return n;
+    }());
+    const size_t off_done = take(sizeof(unsigned) * (nm + nticket_max));
     const size_t off_moms = take(sizeof(MomMatrix) * nm);
     const size_t off_smats = take(sizeof(ScaleMatrix) * nm);
 
@@ -497,10 +559,15 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     const size_t need = cursor;
 
     // ---- arena -----------------------------------------------------------------
-    if (need > arena_bytes) {
+    const int fault = fault_mode();
+    if (need > arena_bytes || fault == FAULT_ALLOC) {
         if (arena_) cudaFree(arena_);
         arena_ = nullptr;
         arena_bytes = 0;
+        if (fault == FAULT_ALLOC) {
+            err = "workspace allocation of " + std::to_string(need) + " bytes failed (injected: MUON_FAULT=alloc)";
+            return MUON_ERR_NO_MEMORY;
+        }
         if (cudaMalloc(&arena_, need) != cudaSuccess) {
             cudaGetLastError();
             err = "workspace allocation of " + std::to_string(need) + " bytes failed";
@@ -540,7 +607,10 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         chained = rounds_per_slot < 16.0;
         if (std::getenv("MUON_CHAIN_LAUNCH")) chained = true;
         if (std::getenv("MUON_SLOT_LAUNCHES")) chained = false;
+        if (fault == FAULT_TIMEOUT) chained = true;  // the injected wait is a chain dependency
     }
+    const unsigned long long wait_ns = wait_limit_ns();
+    size_t nticket = 0;  // tickets handed out so far (one per GEMM launch)
     auto buf_ptr = [&](const Group& g, int b, int z) -> char* {
         return base + g.off[b] + static_cast<size_t>(g.bstride[b]) * z;
     };
@@ -581,8 +651,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         L.bad = d_bad;
         L.status = status;
         L.mat_index_base = 0;
-        L.done = chained ? d_done : nullptr;
-        L.ndone = chained ? nm : 0;
+        L.done = f32 ? nullptr : d_done;
+        L.ndone = f32 ? 0 : static_cast<int>(nm + nticket_max);
         double elems = 0;
         for (int i = 0; i < nm; ++i) elems += static_cast<double>(rq.rows[i]) * rq.cols[i];
         const double per = dtype_size(rq.in_dt) + dtype_size(u_dt) + (rq.is_step ? 2.0 * dtype_size(rq.mom_dt) : 0.0);
@@ -591,11 +661,16 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     }
 
     // ---- steps == 0: elementwise scale / update ---------------------------------
+    // matrices whose schedule has no Newton-Schulz step: X0 itself, applied
+    // by one elementwise launch
     std::vector<ScaleMatrix> smats;
-    if (rq.steps == 0) {
+    bool any_zero_steps = false;
+    for (const Group& g : groups) any_zero_steps |= g.steps == 0;
+    if (any_zero_steps) {
         long long sc = 0;
         for (int i = 0; i < nm; ++i) {
             const Group& g = groups[mat_group[i]];
+            if (g.steps != 0) continue;
             ScaleMatrix s;
             s.u = buf_ptr(g, X0, mat_z[i]);
             s.ldu = g.ldx;
@@ -611,7 +686,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         lr.kind = LaunchRec::SCALE;
         ScaleLaunch& L = lr.sc;
         L.mats = reinterpret_cast<const ScaleMatrix*>(base + off_smats);
-        L.nmats = nm;
+        L.nmats = static_cast<int>(smats.size());
         L.nchunks = sc;
         L.u_dt = u_dt;
         L.out_dt = rq.out_dt;
@@ -633,7 +708,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         std::vector<std::pair<double, int>> cost(nm);
         for (int i = 0; i < nm; ++i) {
             const Group& g = groups[mat_group[i]];
-            cost[i] = {g.slots.empty() ? 0.0 : ns_flops(g.n, g.m, rq.steps, g.form, rq.restart_mask), i};
+            cost[i] = {g.slots.empty() ? 0.0 : ns_flops(g.n, g.m, g.steps, g.form, rq.restart_mask), i};
         }
         std::stable_sort(cost.begin(), cost.end(), [](const std::pair<double, int>& a, const std::pair<double, int>& b) {
             return a.first > b.first;
@@ -904,6 +979,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
             lr.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
             lr.tc.bad = d_bad;
             lr.tc.done = nullptr;
+            lr.tc.ticket = d_done + nm + nticket++;
+            lr.tc.wait_ns = wait_ns;
             lr.tc.status = status;
             // CTA pairs: one cluster of 2 per tile, at most one CTA per SM
             lr.grid = 2 * std::max(1, std::min(lr.tc.ntiles, num_sms / 2));
@@ -918,11 +995,20 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         chain.tc.maps = reinterpret_cast<const CUtensorMap*>(base + off_maps);
         chain.tc.bad = d_bad;
         chain.tc.done = d_done;
+        chain.tc.ticket = d_done + nm + nticket++;
+        chain.tc.wait_ns = wait_ns;
         chain.tc.status = status;
-        // every pair must be co-resident: a tile may wait for any other pair's tiles
+        // one pair per co-resident cluster slot; tiles are claimed in list
+        // order, so pairs that are not resident at once delay nothing
         chain.grid = 2 * std::max(1, std::min(chain.tc.ntiles, max_pairs));
+        if (fault == FAULT_TIMEOUT && !tiles.empty()) tiles[0].need = 0xFFFFFF00u;  // never reached
         launches.push_back(chain);
     }
+    if (nticket > nticket_max) {
+        err = "internal: more GEMM launches than tile tickets";
+        return MUON_ERR_CUDA;
+    }
+    fault_launch_ = fault == FAULT_LAUNCH;
 
     // ---- upload tables -------------------------------------------------------------
     auto up = [&](size_t off, const void* src, size_t bytes) {
@@ -947,6 +1033,10 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
 }
 
 int Plan::run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter, std::string& err) {
+    if (fault_launch_) {
+        err = "kernel launch failed (injected: MUON_FAULT=launch)";
+        return MUON_ERR_CUDA;
+    }
     for (const LaunchRec& lr : launches) {
         if (prof) prof->before(stream);
         cudaError_t e = cudaSuccess;
@@ -961,7 +1051,7 @@ int Plan::run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter,
             return MUON_ERR_CUDA;
         }
         if (launch_counter) ++*launch_counter;
-        if (prof) prof->after(stream, static_cast<int>(lr.kind), lr.flops, lr.bytes);
+        if (prof) prof->after(stream, static_cast<int>(lr.kind), lr.flops, lr.bytes + lr.extra_bytes);
     }
     return MUON_OK;
 }

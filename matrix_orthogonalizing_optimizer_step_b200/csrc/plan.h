@@ -30,6 +30,14 @@ struct PlanRequest {
     int form = FORM_AUTO;
     int steps = 5;
     std::vector<float> coeffs;     // 3*steps
+    // Per-shape schedules: matrix i uses scheds[sched[i]] when sched is not
+    // empty and sched[i] >= 0, else (steps, coeffs) above.
+    struct Schedule {
+        int steps = 0;
+        std::vector<float> coeffs;  // 3*steps
+    };
+    std::vector<Schedule> scheds;
+    std::vector<int> sched;
     unsigned restart_mask = 1u << 2;
     float eps = 1e-7f;
     float mu = 0.95f;
@@ -47,6 +55,7 @@ struct LaunchRec {
     MomLaunch mom{};
     ScaleLaunch sc{};
     double flops = 0, bytes = 0;
+    double extra_bytes = 0;  // the AdamW lane of a hybrid step (momentum launch)
 };
 
 struct ProfileSink {
@@ -64,6 +73,9 @@ class Plan {
     bool same_shape_key(const PlanRequest& req) const;
     // Patch the per-call scalars (mu, nesterov, lr) into the launch records.
     void set_scalars(float mu, int nesterov, float lr, float clip);
+    // Append (or, with null, remove) an AdamW lane to the momentum launch's
+    // grid; `bytes` are its algorithmic HBM bytes (tracing).
+    void set_adamw(const AdamLaunch* adam, double bytes);
     int run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter, std::string& err);
     void release();
     ~Plan() { release(); }
@@ -75,6 +87,7 @@ class Plan {
   private:
     std::vector<long long> key_;
     void* arena_ = nullptr;
+    bool fault_launch_ = false;  // MUON_FAULT=launch: run() fails before its first launch
 };
 
 // Exposed for tests of the host logic: algorithmic FLOPs of one matrix.

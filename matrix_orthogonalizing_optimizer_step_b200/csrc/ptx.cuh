@@ -6,8 +6,9 @@
 
 namespace muon {
 
-// Longest time any wait inside a kernel may spin before it gives up and the
-// kernel reports MUON_ERR_TIMEOUT (nanoseconds of %globaltimer).
+// Default for the longest time any wait inside a kernel may spin before it
+// gives up and the kernel reports MUON_ERR_TIMEOUT (nanoseconds of
+// %globaltimer); each launch carries its own limit.
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -52,15 +53,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait until the phase with the given parity has completed.  Gives up (returns
-// false) when *abort_flag becomes non-zero or after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// false) when *abort_flag becomes non-zero or after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
+        }
+    }
+}
+
+// try_wait with acquire at cluster scope: the waiting thread then sees the
+// memory operations that a thread of another CTA of the cluster released
+// with its arrive (mbar_arrive_cluster) on this barrier.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// mbar_wait with cluster-scope acquire (bounded the same way).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned long long limit_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const unsigned long long t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
         }
     }
 }
@@ -89,6 +120,12 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// 32-bit store to shared memory given by its shared::cluster address (any
+// CTA of the cluster); ordered before a later mbar_arrive_cluster of this thread.
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // ---- cross-CTA dependencies ---------------------------------------------------
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
@@ -111,7 +148,8 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 
 // Wait until *counter >= need (acquire, GPU scope).  Gives up like mbar_wait.
-__device__ __forceinline__ bool wait_counter(const unsigned* counter, unsigned need, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_counter(const unsigned* counter, unsigned need, volatile int* abort_flag,
+                                             unsigned long long limit_ns = kWaitLimitNs) {
     if (ld_acquire_gpu(counter) >= need) return true;
     const unsigned long long t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -119,7 +157,7 @@ __device__ __forceinline__ bool wait_counter(const unsigned* counter, unsigned n
         if (ld_acquire_gpu(counter) >= need) return true;
         if ((it & 15u) == 0u) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
         }
     }
 }

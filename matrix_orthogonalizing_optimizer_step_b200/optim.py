@@ -8,16 +8,19 @@ output classification head.  "工程复现清单": AdamW lr 6e-4, betas
 five Newton-Schulz steps.
 
 This class only keeps the per-parameter state buffers and hands device
-pointers to the library's two fused launches (muon_step for the Muon
-group, muon_adamw_step for the AdamW group); all arithmetic runs in CUDA.
-Gradients may be fp32 or bf16 (one type per group); the installed config's
-gradient and parameter dtypes are set to match for each launch.
+pointers to the library; all arithmetic runs in CUDA.  When both groups use
+one gradient dtype and one parameter dtype, the whole step is ONE hybrid
+call (muon_hybrid_step): the AdamW elements ride in the same grouped
+elementwise launch as the Muon momentum pass, followed by the Newton-Schulz
+launches.  Otherwise each group takes its own call (muon_step,
+muon_adamw_step).  Gradients may be fp32 or bf16; the installed config's
+gradient and parameter dtypes are set to match.
 """
 from __future__ import annotations
 
 import torch
 
-from . import MUON_DTYPE_BF16, MUON_DTYPE_F32, muon_adamw_step, muon_set_config, muon_step
+from . import MUON_DTYPE_BF16, MUON_DTYPE_F32, muon_adamw_step, muon_hybrid_step, muon_set_config, muon_step
 
 _CODE = {torch.float32: MUON_DTYPE_F32, torch.bfloat16: MUON_DTYPE_BF16}
 
@@ -60,6 +63,7 @@ class MuonHybrid(torch.optim.Optimizer):
     @torch.no_grad()
     def step(self, closure=None):
         loss = closure() if closure is not None else None
+        lanes = {}
         for g in self.param_groups:
             ps = [p for p in g["params"] if p.grad is not None]
             if not ps:
@@ -68,35 +72,61 @@ class MuonHybrid(torch.optim.Optimizer):
             pdt = {p.dtype for p in ps}
             if len(gdt) != 1 or len(pdt) != 1 or not (gdt | pdt) <= set(_CODE):
                 raise TypeError("one gradient dtype and one parameter dtype per group, each fp32 or bf16")
-            muon_set_config(grad_dtype=_CODE[gdt.pop()], param_dtype=_CODE[pdt.pop()])
+            dts = (gdt.pop(), pdt.pop())
             if g["kind"] == "muon":
-                W, G, M = [], [], []
-                for p in ps:
-                    st = self.state[p]
-                    if "momentum" not in st:
-                        st["momentum"] = torch.zeros_like(p, dtype=torch.bfloat16)
-                    # conv kernels and other >2-D weights are flattened to 2-D views
-                    W.append(p.view(p.shape[0], -1))
-                    G.append(p.grad.view(p.shape[0], -1))
-                    M.append(st["momentum"].view(p.shape[0], -1))
-                muon_step(W, G, M, mu=g["momentum"], nesterov=g["nesterov"], lr=g["lr"])
+                lanes["muon"] = (g, dts, self._muon_lane(ps))
             else:
-                P, G, M1, M2 = [], [], [], []
-                for p in ps:
-                    st = self.state[p]
-                    if "exp_avg" not in st:
-                        st["exp_avg"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
-                        st["exp_avg_sq"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
-                        st["step"] = 0
-                    st["step"] += 1
-                    P.append(p.view(-1))
-                    G.append(p.grad.view(-1))
-                    M1.append(st["exp_avg"])
-                    M2.append(st["exp_avg_sq"])
-                steps = {self.state[p]["step"] for p in ps}
-                for t in sorted(steps):  # normally one step count for the whole group
-                    idx = [i for i, p in enumerate(ps) if self.state[p]["step"] == t]
-                    muon_adamw_step([P[i] for i in idx], [G[i] for i in idx], [M1[i] for i in idx],
-                                    [M2[i] for i in idx], t, lr=g["lr"], betas=g["betas"], eps=g["eps"],
-                                    weight_decay=g["weight_decay"])
+                lanes["adamw"] = (g, dts, self._adamw_lane(ps))
+        if "muon" in lanes and "adamw" in lanes and lanes["muon"][1] == lanes["adamw"][1] \
+                and len(lanes["adamw"][2]) == 1:
+            # one hybrid call: both lanes in one elementwise launch
+            gm, (gd, pd), (W, G, M) = lanes["muon"]
+            ga, _, by_step = lanes["adamw"]
+            (t, (P, AG, M1, M2)), = by_step.items()
+            muon_set_config(grad_dtype=_CODE[gd], param_dtype=_CODE[pd])
+            muon_hybrid_step(W, G, M, P, AG, M1, M2, t, mu=gm["momentum"], nesterov=gm["nesterov"],
+                             lr=gm["lr"], adam_lr=ga["lr"], betas=ga["betas"], eps=ga["eps"],
+                             weight_decay=ga["weight_decay"])
+            return loss
+        if "muon" in lanes:
+            gm, (gd, pd), (W, G, M) = lanes["muon"]
+            muon_set_config(grad_dtype=_CODE[gd], param_dtype=_CODE[pd])
+            muon_step(W, G, M, mu=gm["momentum"], nesterov=gm["nesterov"], lr=gm["lr"])
+        if "adamw" in lanes:
+            ga, (gd, pd), by_step = lanes["adamw"]
+            muon_set_config(grad_dtype=_CODE[gd], param_dtype=_CODE[pd])
+            for t in sorted(by_step):  # normally one step count for the whole group
+                P, AG, M1, M2 = by_step[t]
+                muon_adamw_step(P, AG, M1, M2, t, lr=ga["lr"], betas=ga["betas"], eps=ga["eps"],
+                                weight_decay=ga["weight_decay"])
         return loss
+
+    def _muon_lane(self, ps):
+        W, G, M = [], [], []
+        for p in ps:
+            st = self.state[p]
+            if "momentum" not in st:
+                st["momentum"] = torch.zeros_like(p, dtype=torch.bfloat16)
+            # conv kernels and other >2-D weights are flattened to 2-D views
+            W.append(p.view(p.shape[0], -1))
+            G.append(p.grad.view(p.shape[0], -1))
+            M.append(st["momentum"].view(p.shape[0], -1))
+        return W, G, M
+
+    def _adamw_lane(self, ps):
+        """{step count: (params, grads, exp_avg, exp_avg_sq)} after advancing
+        every parameter's step count."""
+        by_step = {}
+        for p in ps:
+            st = self.state[p]
+            if "exp_avg" not in st:
+                st["exp_avg"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
+                st["exp_avg_sq"] = torch.zeros(p.numel(), dtype=torch.float32, device=p.device)
+                st["step"] = 0
+            st["step"] += 1
+            lists = by_step.setdefault(st["step"], ([], [], [], []))
+            lists[0].append(p.view(-1))
+            lists[1].append(p.grad.view(-1))
+            lists[2].append(st["exp_avg"])
+            lists[3].append(st["exp_avg_sq"])
+        return by_step

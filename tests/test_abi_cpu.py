@@ -146,3 +146,29 @@ def test_binding_validates_before_calling_the_library():
         mo.muon_adamw_step([torch.zeros(8)], [torch.zeros(9)], [torch.zeros(8)], [torch.zeros(8)], 1)
     with pytest.raises(ValueError):
         mo.muon_adamw_step([torch.zeros(8)], [], [torch.zeros(8)], [torch.zeros(8)], 1)
+
+
+def test_shape_schedule_table(lib):
+    """Per-shape schedules (host-only calls): registration keyed by the short
+    and long side, replacement, lookup, validation and clearing."""
+    mo.muon_reset_config()
+    assert mo.muon_get_shape_coeffs(384, 1536) is None
+    mo.muon_set_shape_coeffs(384, 1536, [(3.0, -4.0, 2.0), (2.0, -1.5, 0.5)])
+    assert mo.muon_get_shape_coeffs(1536, 384) == [(3.0, -4.0, 2.0), (2.0, -1.5, 0.5)]  # transpose shares it
+    mo.muon_set_shape_coeffs(1536, 384, [(1.5, -0.5, 0.0)])                              # replaces it
+    assert mo.muon_get_shape_coeffs(384, 1536) == [(1.5, -0.5, 0.0)]
+    mo.muon_set_shape_coeffs(64, 64, [])                                                 # normalise only
+    assert mo.muon_get_shape_coeffs(64, 64) == []
+    for bad in [(0, 5, [(1, 0, 0)]), (5, -1, [(1, 0, 0)]), (8, 8, [(float("inf"), 0, 0)]),
+                (8, 8, [(1, 0, 0)] * 17)]:
+        with pytest.raises(mo.MuonError) as e:
+            mo.muon_set_shape_coeffs(*bad)
+        assert e.value.code == mo.MUON_ERR_INVALID_ARG
+    mo.muon_clear_shape_coeffs()
+    for k in range(mo.MUON_MAX_SHAPE_SCHEDULES):
+        mo.muon_set_shape_coeffs(8, 8 + k, [(1, 0, 0)])
+    with pytest.raises(mo.MuonError):
+        mo.muon_set_shape_coeffs(8, 1000, [(1, 0, 0)])
+    mo.muon_set_shape_coeffs(8, 8, [(2, 0, 0)])  # replacing an entry is still allowed when full
+    mo.muon_reset_config()  # also clears the table
+    assert mo.muon_get_shape_coeffs(8, 8) is None

@@ -52,18 +52,19 @@ def _shapes():
 
 
 def _make(seed):
+    # fp32 parameters and bf16 momentum: the gather runs once per dtype
     g = torch.Generator().manual_seed(seed)
     P = [torch.randn(s, generator=g) for s in _shapes()]
     G = [torch.randn(s, generator=g) for s in _shapes()]
-    M = [torch.randn(s, generator=g) for s in _shapes()]
+    M = [torch.randn(s, generator=g).to(torch.bfloat16) for s in _shapes()]
     return P, G, M
 
 
 def _standin_step(params, grads, momentum, mu, nesterov, lr):
     # deterministic CPU stand-in for the GPU step (host-logic test only)
     for p, g, m in zip(params, grads, momentum):
-        m.mul_(mu).add_(g)
-        u = g + mu * m if nesterov else m
+        m.copy_(m.float() * mu + g)
+        u = g + mu * m.float() if nesterov else m.float()
         p.sub_(lr * u / (u.norm() + 1e-7))
 
 
@@ -73,12 +74,22 @@ def _worker(rank, world, port, out_q):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
         P, G, M = _make(123)
+        calls = []
+        real = dist.all_gather_into_tensor
+
+        def counting(*a, **k):
+            calls.append(a[0].dtype)
+            return real(*a, **k)
+        dist.all_gather_into_tensor = counting
         owner = sharded.sharded_step(P, G, M, mu=0.9, nesterov=True, lr=0.1, step_fn=_standin_step,
                                      sync_momentum=True)
+        dist.all_gather_into_tensor = real
+        # one collective per dtype (fp32 parameters, bf16 momentum), not one per matrix
+        assert calls == [torch.float32, torch.bfloat16], calls
         import bench
         mx = bench.max_over_ranks(float(rank + 1) * 1.5, world)
         bench.barrier(world)
-        out_q.put((rank, owner, [p.numpy().copy() for p in P], [m.numpy().copy() for m in M], mx))
+        out_q.put((rank, owner, [p.numpy().copy() for p in P], [m.float().numpy().copy() for m in M], mx))
     finally:
         dist.destroy_process_group()
 
@@ -103,7 +114,7 @@ def test_sharded_step_gloo_two_ranks():
     for a, b, ref in zip(P0, P1, P):
         assert (a == b).all() and torch.allclose(torch.from_numpy(a), ref)
     for a, b, ref in zip(M0, M1, M):
-        assert (a == b).all() and torch.allclose(torch.from_numpy(a), ref)
+        assert (a == b).all() and torch.equal(torch.from_numpy(a), ref.float())
     assert mx0 == mx1 == 3.0
 
 

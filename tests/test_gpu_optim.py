@@ -55,3 +55,74 @@ def test_hybrid_step_matches_oracle():
         assert np.max(np.abs(after[name].ravel() - p1)) <= 1e-6 * 1e-3 + 2e-7 * np.max(np.abs(p1)), name
     st, bad = mo.muon_device_status()
     assert st == mo.MUON_OK
+
+
+def _lanes(seed):
+    shapes = [(768, 2304), (768, 768), (3072, 768), (200, 712)]
+    G = [wl.make_single(r, c, seed + 3 * i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, seed + 3 * i + 1, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, seed + 3 * i + 2, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    numels = [50257 * 768, 1024 * 768, 768, 768, 2304, 5, 4099]
+    P = [wl.make_single(1, n, seed + 100 + i, "params", DEV, "f32").view(-1) for i, n in enumerate(numels)]
+    AG = [wl.make_single(1, n, seed + 200 + i, "student_t3", DEV, "bf16", 0.01).view(-1) for i, n in enumerate(numels)]
+    M1 = [torch.zeros(n, device=DEV) for n in numels]
+    M2 = [torch.zeros(n, device=DEV) for n in numels]
+    return (W, G, M), (P, AG, M1, M2)
+
+
+def test_hybrid_call_equals_separate_calls_and_is_one_elementwise_launch():
+    """muon_hybrid_step = muon_step + muon_adamw_step bit for bit, with the
+    AdamW lane inside the momentum launch: one elementwise launch, no AdamW
+    launch, plus the Newton-Schulz launches."""
+    mo.muon_reset_config()
+    (W, G, M), (P, AG, M1, M2) = _lanes(4000)
+    (Wb, _, Mb), (Pb, _, M1b, M2b) = _lanes(4000)
+    for t in (1, 2):
+        mo.muon_step(Wb, G, Mb, mu=0.95, nesterov=True, lr=0.02)
+        mo.muon_adamw_step(Pb, AG, M1b, M2b, t, lr=1e-3)
+    mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, 1, lr=0.02, adam_lr=1e-3)  # builds the plan
+    torch.cuda.synchronize()
+    mo.muon_profile_reset()
+    mo.muon_profile_enable(True)
+    n0 = mo.muon_launch_count()
+    mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, 2, lr=0.02, adam_lr=1e-3)
+    prof = mo.muon_profile_read()
+    mo.muon_profile_enable(False)
+    launched = mo.muon_launch_count() - n0
+    assert prof["momentum_norm"]["launches"] == 1
+    assert prof["adamw"]["launches"] == 0
+    assert launched == 1 + prof["gemm_tc"]["launches"]
+    for x, y in zip(W + M + P + M1 + M2, Wb + Mb + Pb + M1b + M2b):
+        assert torch.equal(x, y)
+    st, _ = mo.muon_device_status()
+    assert st == mo.MUON_OK
+
+
+def test_hybrid_optimizer_issues_one_hybrid_call():
+    mo.muon_reset_config()
+    torch.manual_seed(1)
+    model = Tiny().to(DEV)
+    for i, p in enumerate(model.parameters()):
+        p.grad = wl.make_single(1, p.numel(), 900 + i, "student_t3", DEV, "f32", 0.01).view(p.shape)
+    opt = MuonHybrid(*split_params(model.named_parameters()))
+    opt.step()  # first step builds the plan
+    torch.cuda.synchronize()
+    mo.muon_profile_reset()
+    mo.muon_profile_enable(True)
+    opt.step()
+    prof = mo.muon_profile_read()
+    mo.muon_profile_enable(False)
+    assert prof["momentum_norm"]["launches"] == 1
+    assert prof["adamw"]["launches"] == 0
+
+
+def test_hybrid_argument_error_enqueues_nothing():
+    mo.muon_reset_config()
+    (W, G, M), (P, AG, M1, M2) = _lanes(4100)
+    W0 = [w.clone() for w in W]
+    n0 = mo.muon_launch_count()
+    with pytest.raises(mo.MuonError):
+        mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, 0)  # step 0: invalid AdamW step
+    torch.cuda.synchronize()
+    assert mo.muon_launch_count() == n0
+    assert all(torch.equal(a, b) for a, b in zip(W, W0))

@@ -192,17 +192,38 @@ def test_scale_invariance_bf16():
 
 # ---- aspect-ratio sweep (workload 3), sampled matrices -------------------------
 
+def _sv_gram(x):
+    """Singular values from the eigenvalues of the short-side Gram matrix
+    (the same values as an SVD, far cheaper at these sizes)."""
+    x = np.asarray(x, dtype=np.float64)
+    g = x @ x.T if x.shape[0] <= x.shape[1] else x.T @ x
+    return np.sqrt(np.clip(np.linalg.eigvalsh(g), 0, None))
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("shape", [(2048, 2048), (2048, 8192), (1024, 16384)])
-@pytest.mark.parametrize("form", ["standard", "gram"])
-def test_aspect_sweep_batch16_sampled(shape, form):
+def test_aspect_sweep_batch16_all(shape):
+    """Workload 3 (aspect-ratio sweep, batch 16): every matrix of the batch,
+    standard and Gram forms, against the oracle.  The oracle's two forms agree
+    to 1e-12 in fp64 (pinned on the CPU), so one oracle result per matrix
+    serves both GPU forms."""
     w = wl.WORKLOADS[3]
     idx = [i for i, s in enumerate(w.shapes) if s == shape]
     X = torch.stack([wl.make_matrix(w, i, wl.ROLE_GRAD, device=DEV) for i in idx])
-    Y = _ortho_gpu(X, form)
-    for j in (0, len(idx) - 1):
-        ref = orc.orthogonalize(to64(X[j]), orc.TUNED_COEFFS, 5, form)
-        _check(to64(Y[j]), ref, TOL_BF16_RELF)
+    Ys = {form: to64(_ortho_gpu(X, form)) for form in ("standard", "gram")}
+    n, m = min(shape), max(shape)
+    cheap = "gram" if orc.ns_flops(n, m, 5, "gram") < orc.ns_flops(n, m, 5, "standard") else "standard"
+    worst = {}
+    for j in range(len(idx)):
+        ref = orc.orthogonalize(to64(X[j]), orc.TUNED_COEFFS, 5, cheap)
+        sv_ref = _sv_gram(ref)
+        for form, Y in Ys.items():
+            r = relF(Y[j], ref)
+            sd = float(np.max(np.abs(_sv_gram(Y[j]) - sv_ref)))
+            worst[form] = max(worst.get(form, 0.0), r)
+            assert r <= TOL_BF16_RELF, (form, j, r)
+            assert sd <= TOL_SIGMA, (form, j, sd)
+    print(shape, "worst relF", worst)
 
 
 def test_fitted_per_shape_schedule():

@@ -1,0 +1,185 @@
+"""Failure paths and scheduling robustness of the GPU path.
+
+* Host-side fault injection (MUON_FAULT=alloc | launch): the call returns
+  MUON_ERR_NO_MEMORY / MUON_ERR_CUDA, launches no kernel and leaves every
+  caller tensor untouched; the next normal call succeeds with parity.
+* A bounded device wait that runs out (MUON_FAULT=timeout gives the first
+  tile of a chained launch a dependency count that no tile will reach, with
+  a short MUON_WAIT_LIMIT_MS): the kernel gives up, the status word reads
+  MUON_ERR_TIMEOUT, the context stays usable and the next normal call
+  returns MUON_OK with parity.  Nothing faults, traps or hangs the GPU.
+* The chained launch while other work holds SMs: tiles are claimed in list
+  order, so the step completes and equals an unloaded run bit for bit.
+* Calls alternating between two streams on independent buffers: the
+  library's shared workspace is ordered across the streams.
+"""
+import time
+
+import numpy as np
+import pytest
+import torch
+
+import matrix_orthogonalizing_optimizer_step_b200 as mo
+from matrix_orthogonalizing_optimizer_step_b200 import workloads as wl
+from oracle import muon_oracle as orc
+from tests._util import TOL_BF16_RELF, relF, to64
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+SHAPES = [(256, 768), (768, 256), (200, 200), (136, 520)]
+
+
+@pytest.fixture(autouse=True)
+def _fresh(monkeypatch):
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES"):
+        monkeypatch.delenv(k, raising=False)
+    mo.muon_reset_config()
+    mo.muon_release_workspace()
+    yield
+    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES"):
+        monkeypatch.delenv(k, raising=False)
+    mo.muon_release_workspace()
+    st, bad = mo.muon_device_status()
+    assert st == mo.MUON_OK, (mo.STATUS_NAMES.get(st), bad)
+    mo.muon_reset_config()
+
+
+def _make_set(shapes, seed):
+    G = [wl.make_single(r, c, seed + 3 * i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, seed + 3 * i + 1, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, seed + 3 * i + 2, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    return W, G, M
+
+
+def _step_and_check(shapes, seed, lr=0.1):
+    """A normal step that must succeed and match the oracle."""
+    W, G, M = _make_set(shapes, seed)
+    W64, G64, M64 = [to64(t) for t in W], [to64(t) for t in G], [to64(t) for t in M]
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=lr)
+    st, bad = mo.muon_device_status()
+    assert st == mo.MUON_OK, (mo.STATUS_NAMES.get(st), bad)
+    for i in range(len(shapes)):
+        _, _, O = orc.muon_step(W64[i], G64[i], M64[i], 0.95, True, lr, form="standard")
+        assert relF((W64[i] - to64(W[i])) / lr, O) <= TOL_BF16_RELF, (shapes[i],)
+
+
+@pytest.mark.parametrize("fault,code", [("alloc", mo.MUON_ERR_NO_MEMORY), ("launch", mo.MUON_ERR_CUDA)])
+def test_injected_host_fault_enqueues_nothing(fault, code, monkeypatch):
+    W, G, M = _make_set(SHAPES, 10)
+    W0, M0 = [t.clone() for t in W], [t.clone() for t in M]
+    torch.cuda.synchronize()
+    monkeypatch.setenv("MUON_FAULT", fault)
+    n0 = mo.muon_launch_count()
+    with pytest.raises(mo.MuonError) as e:
+        mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.1)
+    assert e.value.code == code
+    assert fault in str(e.value)
+    torch.cuda.synchronize()
+    assert mo.muon_launch_count() == n0
+    for x, y in zip(W + M, W0 + M0):
+        assert torch.equal(x, y)
+    monkeypatch.delenv("MUON_FAULT")
+    _step_and_check(SHAPES, 20)
+
+
+def test_injected_alloc_failure_adamw(monkeypatch):
+    P = [wl.make_single(1, n, 40 + i, "params", DEV, "f32").view(-1) for i, n in enumerate([4096, 1000])]
+    G = [torch.ones_like(p, dtype=torch.bfloat16) for p in P]
+    M1 = [torch.zeros_like(p) for p in P]
+    M2 = [torch.zeros_like(p) for p in P]
+    P0 = [p.clone() for p in P]
+    monkeypatch.setenv("MUON_FAULT", "alloc")
+    n0 = mo.muon_launch_count()
+    with pytest.raises(mo.MuonError) as e:
+        mo.muon_adamw_step(P, G, M1, M2, 1)
+    assert e.value.code == mo.MUON_ERR_NO_MEMORY
+    torch.cuda.synchronize()
+    assert mo.muon_launch_count() == n0
+    assert all(torch.equal(p, q) for p, q in zip(P, P0))
+    monkeypatch.delenv("MUON_FAULT")
+    mo.muon_adamw_step(P, G, M1, M2, 1)
+    torch.cuda.synchronize()
+    assert not torch.equal(P[0], P0[0])
+
+
+def test_bounded_wait_runs_out_and_context_stays_usable(monkeypatch):
+    monkeypatch.setenv("MUON_FAULT", "timeout")
+    monkeypatch.setenv("MUON_WAIT_LIMIT_MS", "50")
+    W, G, M = _make_set(SHAPES, 30)
+    t0 = time.perf_counter()
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.1)  # enqueued: returns OK
+    st, bad = mo.muon_device_status()                       # synchronises
+    elapsed = time.perf_counter() - t0
+    assert st == mo.MUON_ERR_TIMEOUT, mo.STATUS_NAMES.get(st)
+    assert elapsed < 20.0  # every wait gave up after its 50 ms bound
+    # the status word was cleared by the read; a normal call works again
+    monkeypatch.delenv("MUON_FAULT")
+    monkeypatch.delenv("MUON_WAIT_LIMIT_MS")
+    mo.muon_release_workspace()
+    _step_and_check(SHAPES, 40)
+
+
+def test_chained_launch_under_sm_contention(monkeypatch):
+    """Other kernels hold SMs while the chained step starts (a side stream of
+    large matmuls, a few hundred ms of work): not every CTA pair of the launch
+    is resident at once.  The step must complete without a timeout and equal
+    the unloaded run bit for bit (a tile's arithmetic does not depend on which
+    pair computes it)."""
+    monkeypatch.setenv("MUON_CHAIN_LAUNCH", "1")
+    shapes = [(768, 2304), (768, 768), (768, 3072), (3072, 768)] * 3
+    W, G, M = _make_set(shapes, 50)
+    Wr, Mr = [t.clone() for t in W], [t.clone() for t in M]
+    mo.muon_step(Wr, G, Mr, mu=0.95, nesterov=True, lr=0.02)
+    st, _ = mo.muon_device_status()
+    assert st == mo.MUON_OK
+    A = torch.randn(8192, 8192, device=DEV, dtype=torch.bfloat16)
+    side = torch.cuda.Stream(DEV)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        for _ in range(300):
+            B = A @ A
+    mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.02)
+    torch.cuda.synchronize()
+    del B
+    st, bad = mo.muon_device_status()
+    assert st == mo.MUON_OK, (mo.STATUS_NAMES.get(st), bad)
+    for x, y in zip(W + M, Wr + Mr):
+        assert torch.equal(x, y)
+
+
+def test_calls_alternating_streams():
+    """Independent batches orthogonalised alternately on two streams with no
+    ordering between the caller's streams: every call reuses the library's
+    workspace (a different buffer means a new plan), and the library orders
+    each use after the previous one, so the results equal a serial run."""
+    xs = [torch.stack([wl.make_single(1024, 4096, 60 + 8 * k + j, "gaussian", DEV, "bf16") for j in range(4)])
+          for k in range(4)]
+    ref = [x.clone() for x in xs]
+    for x in ref:
+        mo.muon_orthogonalize(x, steps=5, mode="gram")
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(DEV), torch.cuda.Stream(DEV)]
+    got = [x.clone() for x in xs]
+    torch.cuda.synchronize()
+    for rnd in range(2):
+        # buffer k always runs on stream k % 2, so each buffer's own calls are
+        # ordered by its stream; only the workspace is shared across streams
+        for k, x in enumerate(got):
+            with torch.cuda.stream(streams[k % 2]):
+                mo.muon_orthogonalize(x, steps=5, mode="gram")
+        if rnd == 0:
+            # round 0 equals the serial reference
+            torch.cuda.synchronize()
+            for a, b in zip(got, ref):
+                assert torch.equal(a, b)
+    torch.cuda.synchronize()
+    # round 1 orthogonalised the outputs again: compare with the same on one stream
+    for x in ref:
+        mo.muon_orthogonalize(x, steps=5, mode="gram")
+    torch.cuda.synchronize()
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    st, _ = mo.muon_device_status()
+    assert st == mo.MUON_OK
+    assert np.all(np.isfinite(to64(got[0])))

@@ -34,12 +34,14 @@
 // dependency waits of one matrix are filled with other matrices' tiles.
 //
 // Tiles are claimed, in list order, from a global ticket by the leader CTA's
-// producer, one tile ahead of the one it is loading, and handed to every role
-// of both CTAs through a small ring of tile indices in shared memory.  A tile
-// that waits on earlier tiles therefore only ever waits on tiles that running
-// pairs have claimed: the launch makes progress however many of its pairs
-// are resident (other kernels may hold SMs), and the dynamic order also
-// balances tiles of unequal K across pairs.
+// producer and handed to every role of both CTAs through a small ring of tile
+// records in shared memory (the producer publishes a tile as it starts loading
+// it; the claim of the next tile is issued then and only consumed once the
+// current tile's loads are under way, so its latency is hidden).  A tile that
+// waits on earlier tiles therefore only ever waits on tiles that running pairs
+// have claimed: the launch makes progress however many of its pairs are
+// resident (other kernels may hold SMs), and the dynamic order also balances
+// tiles of unequal K across pairs.
 //
 // Every wait is bounded: on expiry the kernel records a timeout in the device
 // status word, drains its own copies and MMAs, frees TMEM and exits.
@@ -68,47 +70,57 @@ constexpr uint32_t TMEM_COLS = 512;  // 2 accumulators x 256 fp32 columns
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
 constexpr int STORE_BOX_BYTES = 64 * 32;  // one TMA store box: 32 rows of 64 bytes
 constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per epilogue warp
-constexpr int SCHED = 8;  // depth of the tile-index ring
+constexpr int SCHED = 8;  // depth of the tile-record ring
 // readers of every ring slot: the leader's MMA thread, the peer's producer,
 // and the epilogue warps of both CTAs
 constexpr uint32_t SCHED_READERS = 2 + 2 * EPI_WARPS;
-constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 512 /*barriers, ring*/;
+constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 1024 /*barriers, ring*/;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
 
+// A ring slot: the raw 32-byte tile record (TcTile), or kRingEnd in its
+// first word once the launch's tiles are exhausted.
+struct RingRec {
+    uint4 a, b;
+};
+constexpr unsigned kRingEnd = 0xFFFFFFFFu;
+
 struct Shared {
+    RingRec ring[SCHED];     // claimed tiles' records (leader's producer writes both CTAs')
     uint64_t full[STAGES];   // leader: both CTAs' operand bytes landed
     uint64_t empty[STAGES];  // each CTA: its slot may be refilled (leader's MMA commit)
     uint64_t tfull[2];       // each CTA: accumulator ready (leader's MMA commit)
     uint64_t tempty[2];      // leader: all 2 x EPI_WARPS epilogue warps drained the accumulator
-    uint64_t sfull[SCHED];   // each CTA: ring slot holds a claimed tile index (leader's producer)
+    uint64_t sfull[SCHED];   // each CTA: ring slot holds a record (leader's producer)
     uint64_t sempty[SCHED];  // leader: every reader of both CTAs has read the ring slot
     uint64_t drain;
-    int sched[SCHED];        // claimed tile indices; ntiles: no more tiles
     uint32_t tmem_base;
     int abort;
 };
-static_assert(sizeof(Shared) <= 512, "barrier area");
+static_assert(sizeof(Shared) <= 1024, "barrier area");
 
 // Symmetric operands are stored as upper 256 x 256 tiles: the 64-wide K slice
 // kb of the 256-row block `blk` lies in a lower (unstored) tile when blk > kb/4.
 __device__ __forceinline__ bool slice_is_lower(int blk, int kb) { return blk > (kb * BK) / BN; }
 
 // Tile records never change during a launch: read-only path, two 16-byte loads.
-__device__ __forceinline__ TcTile load_tile(const TcTile* tiles, int t) {
+__device__ __forceinline__ RingRec load_tile_raw(const TcTile* tiles, int t) {
     const uint4* p = reinterpret_cast<const uint4*>(tiles + t);
-    const uint4 a = __ldg(p), b = __ldg(p + 1);
+    return RingRec{__ldg(p), __ldg(p + 1)};
+}
+
+__device__ __forceinline__ TcTile decode_tile(const RingRec& r) {
     TcTile x;
-    x.problem = a.x;
-    x.bibj = a.y;
-    x.mat = a.z;
-    x.need = a.w;
-    x.kf = b.x;
-    x.a_map = static_cast<unsigned short>(b.y & 0xFFFFu);
-    x.b_map = static_cast<unsigned short>(b.y >> 16);
-    x.a_map_t = static_cast<unsigned short>(b.z & 0xFFFFu);
-    x.b_map_t = static_cast<unsigned short>(b.z >> 16);
-    x.a_z = static_cast<unsigned short>(b.w & 0xFFFFu);
-    x.b_z = static_cast<unsigned short>(b.w >> 16);
+    x.problem = r.a.x;
+    x.bibj = r.a.y;
+    x.mat = r.a.z;
+    x.need = r.a.w;
+    x.kf = r.b.x;
+    x.a_map = static_cast<unsigned short>(r.b.y & 0xFFFFu);
+    x.b_map = static_cast<unsigned short>(r.b.y >> 16);
+    x.a_map_t = static_cast<unsigned short>(r.b.z & 0xFFFFu);
+    x.b_map_t = static_cast<unsigned short>(r.b.z >> 16);
+    x.a_z = static_cast<unsigned short>(r.b.w & 0xFFFFu);
+    x.b_z = static_cast<unsigned short>(r.b.w >> 16);
     return x;
 }
 
@@ -117,25 +129,20 @@ __device__ __forceinline__ void record_timeout(Shared* sh, DeviceStatus* st) {
     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
 }
 
-// Next unclaimed tile of the launch (ntiles once the list is exhausted).
-__device__ __forceinline__ int claim_tile(const TcLaunch& L) {
-    const unsigned t = atomicAdd(L.ticket, 1u);
-    return t < static_cast<unsigned>(L.ntiles) ? static_cast<int>(t) : L.ntiles;
-}
-
-// Writer side of the tile-index ring (the leader's producer): publish t in
+// Writer side of the tile ring (the leader's producer): publish a record in
 // the same slot of both CTAs' rings once every reader has read that slot's
-// previous value.  False when that wait ran out.
+// previous record.  False when that wait ran out.
 struct RingWriter {
     int slot = 0;
     uint32_t phase = 0;
-    __device__ bool push(Shared* sh, int t, volatile int* abort_flag, unsigned long long limit) {
+    __device__ bool push(Shared* sh, const RingRec& rec, volatile int* abort_flag, unsigned long long limit) {
         if (!mbar_wait_cluster(&sh->sempty[slot], phase ^ 1u, abort_flag, limit)) return false;
-        const uint32_t v = smem_u32(&sh->sched[slot]), b = smem_u32(&sh->sfull[slot]);
+        const uint32_t v = smem_u32(&sh->ring[slot]), b = smem_u32(&sh->sfull[slot]);
 #pragma unroll
         for (uint32_t r = 0; r < 2; ++r) {
-            st_shared_cluster_u32(map_to_cta(v, r), static_cast<uint32_t>(t));
-            mbar_arrive_cluster(map_to_cta(b, r));  // release: the index is visible first
+            st_shared_cluster_v4(map_to_cta(v, r), rec.a);
+            st_shared_cluster_v4(map_to_cta(v + 16, r), rec.b);
+            mbar_arrive_cluster(map_to_cta(b, r));  // release: the record is visible first
         }
         if (++slot == SCHED) {
             slot = 0;
@@ -145,21 +152,34 @@ struct RingWriter {
     }
 };
 
-// Reader side: the next published tile index, or -1 when the wait ran out.
+// Reader side: the next published record (false when the wait ran out).
 struct RingReader {
     int slot = 0;
     uint32_t phase = 0;
-    __device__ int pop(Shared* sh, volatile int* abort_flag, unsigned long long limit) {
-        if (!mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit)) return -1;
-        const int t = *reinterpret_cast<volatile int*>(&sh->sched[slot]);
+    __device__ bool pop(Shared* sh, RingRec& rec, volatile int* abort_flag, unsigned long long limit) {
+        if (!mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit)) return false;
+        const volatile uint4* p = reinterpret_cast<const volatile uint4*>(&sh->ring[slot]);
+        rec.a = make_uint4(p[0].x, p[0].y, p[0].z, p[0].w);
+        rec.b = make_uint4(p[1].x, p[1].y, p[1].z, p[1].w);
         mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sempty[slot]), 0));  // read: the slot is free
         if (++slot == SCHED) {
             slot = 0;
             phase ^= 1u;
         }
-        return t;
+        return true;
+    }
+    // The next record if it is already published, without consuming it (its
+    // slot cannot be rewritten before this reader has popped it).
+    __device__ bool peek(Shared* sh, RingRec& rec) {
+        if (!mbar_try_wait_cluster(&sh->sfull[slot], phase)) return false;
+        const volatile uint4* p = reinterpret_cast<const volatile uint4*>(&sh->ring[slot]);
+        rec.a = make_uint4(p[0].x, p[0].y, p[0].z, p[0].w);
+        rec.b = make_uint4(p[1].x, p[1].y, p[1].z, p[1].w);
+        return true;
     }
 };
+
+__device__ __forceinline__ RingRec end_rec() { return RingRec{make_uint4(kRingEnd, 0, 0, 0), make_uint4(0, 0, 0, 0)}; }
 
 __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t rank) {
     volatile int* abort_flag = &sh->abort;
@@ -173,33 +193,35 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     unsigned seen_mat = ~0u, seen_done = 0;  // counters only grow within a launch
     RingWriter wr;
     RingReader rd;
-    // The leader claims tiles and publishes them to both CTAs' rings; the
-    // peer reads them.  -1: a wait ran out.
-    auto next_tile = [&]() -> int {
-        if (leader) {
-            const int t = claim_tile(L);
-            return wr.push(sh, t, abort_flag, lim) ? t : -1;
-        }
-        return rd.pop(sh, abort_flag, lim);
-    };
-    // The next tile is claimed (and its record fetched) while the current one
-    // is loaded, and its dependency and tensor maps are acquired right after
-    // the current tile's last fill is issued (the slices still queued in the
-    // ring hide the wait), so consecutive tiles follow each other without a
-    // gap in the fills.
+    // The leader claims tiles and publishes their records to both CTAs'
+    // rings as it starts loading them; the peer reads them.  The claim of the
+    // next tile is issued when the current one is published and consumed two
+    // K slices into its loads, and the next record is fetched then: neither
+    // latency sits between two tiles.  The next tile's dependency and tensor
+    // maps are acquired right after the current tile's last fill is issued
+    // (the slices still queued hide the wait).
     bool early = false;  // the current tile's dependency was acquired early
-    int t = next_tile();
-    TcTile nxt;
-    if (t < 0) ok = false;
-    if (ok && t < L.ntiles) nxt = load_tile(L.tiles, t);
-    while (ok && t < L.ntiles) {
-        const TcTile tile = nxt;
-        const int tn = next_tile();
-        if (tn < 0) {
+    RingRec cur;
+    if (leader) {
+        const unsigned t0 = atomicAdd(L.ticket, 1u);
+        cur = t0 < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(t0)) : end_rec();
+    }
+    while (ok) {
+        if (leader) {
+            if (!wr.push(sh, cur, abort_flag, lim)) {
+                ok = false;
+                break;
+            }
+        } else if (!rd.pop(sh, cur, abort_flag, lim)) {
             ok = false;
             break;
         }
-        if (tn < L.ntiles) nxt = load_tile(L.tiles, tn);
+        if (cur.a.x == kRingEnd) break;
+        const TcTile tile = decode_tile(cur);
+        unsigned claim = 0;
+        if (leader) claim = atomicAdd(L.ticket, 1u);
+        RingRec nxt_rec;
+        bool have_next = false;
         // operands produced by earlier chain slots of the same matrix
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
             if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag, lim)) {
@@ -265,8 +287,15 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 stage = 0;
                 phase ^= 1u;
             }
+            if (leader && !have_next && (kb >= 2 || kb == nk - 1)) {
+                nxt_rec = claim < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(claim))
+                                                                  : end_rec();
+                have_next = true;
+            }
         }
-        if (ok && tn < L.ntiles) {
+        if (ok && !leader) have_next = rd.peek(sh, nxt_rec);  // published already?
+        if (ok && have_next && nxt_rec.a.x != kRingEnd) {
+            const TcTile nxt = decode_tile(nxt_rec);
             if (nxt.need && !(nxt.mat == seen_mat && nxt.need <= seen_done))
                 early = ld_acquire_gpu(L.done + nxt.mat) >= nxt.need;
             const unsigned nfl = nxt.kf >> 24;
@@ -281,7 +310,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 last_b = nxt.b_map;
             }
         }
-        t = tn;
+        if (leader) cur = have_next ? nxt_rec : end_rec();
     }
     if (!ok) record_timeout(sh, L.status);
     // Drain (leader): the last fills of every stage must have landed before
@@ -309,18 +338,14 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     bool issued_any = false;
     const uint32_t tiles_base = smem_u32(tiles_smem);
     RingReader rd;
-    int t = rd.pop(sh, abort_flag, lim);
-    if (t < 0) ok = false;
-    TcTile nxt;
-    if (ok && t < L.ntiles) nxt = load_tile(L.tiles, t);
-    while (ok && t < L.ntiles) {
-        const TcTile tile = nxt;
-        const int tn = rd.pop(sh, abort_flag, lim);  // claimed ahead by the producer
-        if (tn < 0) {
+    while (ok) {
+        RingRec rec;
+        if (!rd.pop(sh, rec, abort_flag, lim)) {  // published as the producer starts its loads
             ok = false;
             break;
         }
-        if (tn < L.ntiles) nxt = load_tile(L.tiles, tn);  // in flight during this tile
+        if (rec.a.x == kRingEnd) break;
+        const TcTile tile = decode_tile(rec);
         const int K = static_cast<int>(tile.kf & kTileMaxK);
         const unsigned fl = tile.kf >> 24;
         const int a_mn = (fl & TILE_A_MN) ? 1 : 0, b_mn = (fl & TILE_B_MN) ? 1 : 0;
@@ -368,7 +393,6 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             acc = 0;
             acc_phase ^= 1u;
         }
-        t = tn;
     }
     if (!ok) {
         record_timeout(sh, L.status);
@@ -397,21 +421,24 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     // this lane's 64-byte row of a store box, 16-byte units swizzled (64-byte mode)
     const uint32_t row_off = static_cast<uint32_t>(lane) * 64;
     const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
-    // lane 0 reads the tile-index ring for the warp (one reader per warp)
+    // lane 0 reads the tile ring for the warp (one reader per warp) and
+    // passes the record's first half (problem, position, matrix, dependency)
     RingReader rd;
-    auto next_tile = [&]() -> int {
-        int v = 0;
-        if (lane == 0) v = rd.pop(sh, abort_flag, lim);
-        return __shfl_sync(0xffffffffu, v, 0);
-    };
-    int t = next_tile();
-    while (t >= 0 && t < L.ntiles) {
-        const int tn = next_tile();  // claimed ahead by the producer
-        if (tn < 0) {
-            if (lane == 0) record_timeout(sh, L.status);
+    bool timed_out = false;
+    while (true) {
+        RingRec rec;
+        int got_rec = 1;
+        if (lane == 0) got_rec = rd.pop(sh, rec, abort_flag, lim) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, got_rec, 0)) {
+            timed_out = true;
             break;
         }
-        const TcTile tile = load_tile(L.tiles, t);
+        TcTile tile;
+        tile.problem = __shfl_sync(0xffffffffu, rec.a.x, 0);
+        tile.bibj = __shfl_sync(0xffffffffu, rec.a.y, 0);
+        tile.mat = __shfl_sync(0xffffffffu, rec.a.z, 0);
+        tile.need = __shfl_sync(0xffffffffu, rec.a.w, 0);
+        if (tile.problem == kRingEnd) break;
         // Local copies: the epilogue stores to global memory, so fields read
         // through a reference into the problem table would be reloaded after
         // every store (the compiler cannot rule out aliasing).
@@ -539,9 +566,8 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             acc = 0;
             acc_phase ^= 1u;
         }
-        t = tn;
     }
-    if (t < 0 && lane == 0) record_timeout(sh, L.status);
+    if (timed_out && lane == 0) record_timeout(sh, L.status);
     // the staging boxes must stay valid until every store has read them
     if (lane == 0) bulk_wait_all();
     __syncwarp();

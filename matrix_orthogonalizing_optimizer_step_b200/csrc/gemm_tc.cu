@@ -35,9 +35,10 @@
 //
 // Tiles are claimed, in list order, from a global ticket by the leader CTA's
 // producer and handed to every role of both CTAs through a small ring of tile
-// records in shared memory (the producer publishes a tile as it starts loading
-// it; the claim of the next tile is issued then and only consumed once the
-// current tile's loads are under way, so its latency is hidden).  A tile that
+// records in shared memory.  The claim of the next tile is issued as the
+// current one starts, its record fetched two K slices into the current tile's
+// loads and published two slices later, so neither latency sits between two
+// tiles and the peer CTA's producer knows its next tile before it gets there.  A tile that
 // waits on earlier tiles therefore only ever waits on tiles that running pairs
 // have claimed: the launch makes progress however many of its pairs are
 // resident (other kernels may hold SMs), and the dynamic order also balances
@@ -194,25 +195,21 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     RingWriter wr;
     RingReader rd;
     // The leader claims tiles and publishes their records to both CTAs'
-    // rings as it starts loading them; the peer reads them.  The claim of the
-    // next tile is issued when the current one is published and consumed two
-    // K slices into its loads, and the next record is fetched then: neither
-    // latency sits between two tiles.  The next tile's dependency and tensor
-    // maps are acquired right after the current tile's last fill is issued
-    // (the slices still queued hide the wait).
+    // rings one tile ahead; the peer reads them.  The claim of the next tile
+    // is issued when the current one starts and consumed two K slices into
+    // its loads, where the next record is fetched; it is published two slices
+    // later.  The next tile's dependency and tensor maps are acquired right
+    // after the current tile's last fill is issued (the slices still queued
+    // hide the wait).
     bool early = false;  // the current tile's dependency was acquired early
     RingRec cur;
     if (leader) {
         const unsigned t0 = atomicAdd(L.ticket, 1u);
         cur = t0 < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(t0)) : end_rec();
+        if (!wr.push(sh, cur, abort_flag, lim)) ok = false;
     }
     while (ok) {
-        if (leader) {
-            if (!wr.push(sh, cur, abort_flag, lim)) {
-                ok = false;
-                break;
-            }
-        } else if (!rd.pop(sh, cur, abort_flag, lim)) {
+        if (!leader && !rd.pop(sh, cur, abort_flag, lim)) {
             ok = false;
             break;
         }
@@ -221,7 +218,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
         unsigned claim = 0;
         if (leader) claim = atomicAdd(L.ticket, 1u);
         RingRec nxt_rec;
-        bool have_next = false;
+        bool have_next = false, pushed = false;
         // operands produced by earlier chain slots of the same matrix
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
             if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag, lim)) {
@@ -292,6 +289,13 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                                                                   : end_rec();
                 have_next = true;
             }
+            if (leader && have_next && !pushed && (kb >= 4 || kb == nk - 1)) {
+                if (!wr.push(sh, nxt_rec, abort_flag, lim)) {
+                    ok = false;
+                    break;
+                }
+                pushed = true;
+            }
         }
         if (ok && !leader) have_next = rd.peek(sh, nxt_rec);  // published already?
         if (ok && have_next && nxt_rec.a.x != kRingEnd) {
@@ -310,7 +314,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 last_b = nxt.b_map;
             }
         }
-        if (leader) cur = have_next ? nxt_rec : end_rec();
+        if (leader) cur = nxt_rec;  // pushed in the K loop (ok) or not needed (timed out)
     }
     if (!ok) record_timeout(sh, L.status);
     // Drain (leader): the last fills of every stage must have landed before

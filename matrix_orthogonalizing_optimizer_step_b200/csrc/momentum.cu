@@ -81,13 +81,16 @@ __device__ __forceinline__ T block_sum(T v, T* red) {
     return r;  // valid in thread 0
 }
 
-template <bool G_F32, int MOM, bool U_F32, bool CLIP>
+// HYBRID: the grid also carries the AdamW lane's chunks (after the Muon
+// chunks).  A separate instance, so that the plain Muon step keeps the small
+// register footprint (and the occupancy) of the momentum pass alone.
+template <bool G_F32, int MOM, bool U_F32, bool CLIP, bool HYBRID>
 __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch L) {
     __shared__ float red_f[kThreads / 32];
     __shared__ double red_d[kThreads / 32];
     __shared__ int is_last;
     const long long chunk = blockIdx.x;
-    if (chunk >= L.nchunks) {
+    if (HYBRID && chunk >= L.nchunks) {
         // hybrid step: the AdamW lane's chunks follow the Muon chunks
         if (L.adam.p_dt == DT_F32)
             adamw_chunk<true, G_F32>(L.adam, chunk - L.nchunks);
@@ -217,39 +220,44 @@ __global__ void __launch_bounds__(kThreads) scale_apply_kernel(const ScaleLaunch
 
 }  // namespace
 
-template <bool CLIP>
+template <bool CLIP, bool HYBRID>
 static cudaError_t launch_step(const MomLaunch& L, dim3 grid, bool gf, cudaStream_t stream) {
     if (gf) {
         if (L.mom_dt == DT_F32)
-            momentum_norm_kernel<true, MOM_F32, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<true, MOM_F32, false, CLIP, HYBRID><<<grid, kThreads, 0, stream>>>(L);
         else
-            momentum_norm_kernel<true, MOM_BF16, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<true, MOM_BF16, false, CLIP, HYBRID><<<grid, kThreads, 0, stream>>>(L);
     } else {
         if (L.mom_dt == DT_F32)
-            momentum_norm_kernel<false, MOM_F32, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<false, MOM_F32, false, CLIP, HYBRID><<<grid, kThreads, 0, stream>>>(L);
         else
-            momentum_norm_kernel<false, MOM_BF16, false, CLIP><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<false, MOM_BF16, false, CLIP, HYBRID><<<grid, kThreads, 0, stream>>>(L);
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream) {
     if (L.nchunks <= 0) return cudaSuccess;
-    if (L.adam.ntensors > 0 && (!L.has_momentum || L.adam.g_dt != L.in_dt)) return cudaErrorInvalidValue;
-    const dim3 grid(static_cast<unsigned>(L.nchunks + (L.adam.ntensors > 0 ? L.adam.nchunks : 0)));
+    const bool hybrid = L.adam.ntensors > 0;
+    if (hybrid && (!L.has_momentum || L.adam.g_dt != L.in_dt)) return cudaErrorInvalidValue;
+    const dim3 grid(static_cast<unsigned>(L.nchunks + (hybrid ? L.adam.nchunks : 0)));
     const bool gf = L.in_dt == DT_F32, uf = L.u_dt == DT_F32;
     if (!L.has_momentum) {
         if (gf && uf)
-            momentum_norm_kernel<true, MOM_NONE, true, false><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<true, MOM_NONE, true, false, false><<<grid, kThreads, 0, stream>>>(L);
         else if (!gf && !uf)
-            momentum_norm_kernel<false, MOM_NONE, false, false><<<grid, kThreads, 0, stream>>>(L);
+            momentum_norm_kernel<false, MOM_NONE, false, false, false><<<grid, kThreads, 0, stream>>>(L);
         else
             return cudaErrorInvalidValue;
         return cudaGetLastError();
     }
     if (uf) return cudaErrorInvalidValue;
-    if (L.clip > 0.f) return launch_step<true>(L, grid, gf, stream);
-    return launch_step<false>(L, grid, gf, stream);
+    if (hybrid) {
+        if (L.clip > 0.f) return launch_step<true, true>(L, grid, gf, stream);
+        return launch_step<false, true>(L, grid, gf, stream);
+    }
+    if (L.clip > 0.f) return launch_step<true, false>(L, grid, gf, stream);
+    return launch_step<false, false>(L, grid, gf, stream);
 }
 
 cudaError_t launch_scale_apply(const ScaleLaunch& L, cudaStream_t stream) {

@@ -917,8 +917,17 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                         const unsigned pi = static_cast<unsigned>(tprobs.size());
                         tprobs.push_back(p);
                         const int tm = (M + tile_m - 1) / tile_m, tn = (N + tile_n - 1) / tile_n;
-                        for (int bi = 0; bi < tm; ++bi)
-                            for (int bj = 0; bj < tn; ++bj) {
+                        // Tile order within a problem: consecutive tiles (the ones
+                        // the pairs work on at once) should share the panels of
+                        // the big operand.  A non-transposed apply (n x n factor
+                        // times the n x m X) is listed column by column, so the
+                        // pairs at work share one or two column panels of X and
+                        // the whole small factor; every other product row by row.
+                        const bool col_major = op.kind == OP_APPLY && !g.trans;
+                        const int outer = col_major ? tn : tm, inner = col_major ? tm : tn;
+                        for (int o = 0; o < outer; ++o)
+                            for (int i2 = 0; i2 < inner; ++i2) {
+                                const int bi = col_major ? i2 : o, bj = col_major ? o : i2;
                                 if (op.sym && bi * tile_m > bj * tile_n + tile_n - 1) continue;
                                 TcTile tt;
                                 std::memset(&tt, 0, sizeof(tt));

@@ -11,6 +11,7 @@
 // 64-wide K slice this moves 32 KB of operands for 4.2 MFLOP, a third less
 // than a single-CTA 128 x 256 tile.
 //
+//   warp 10     tile scheduler (leader CTA): claims tiles, publishes records
 //   warp 0      TMA producer (both CTAs): 64-wide K slices of its halves of A
 //               and B into a 5-stage ring (128-byte swizzle, no multicast);
 //               the transaction bytes of both CTAs land on the leader's barrier
@@ -33,16 +34,16 @@
 // per-matrix completion counter; matrices progress independently, so the
 // dependency waits of one matrix are filled with other matrices' tiles.
 //
-// Tiles are claimed, in list order, from a global ticket by the leader CTA's
-// producer and handed to every role of both CTAs through a small ring of tile
-// records in shared memory.  The claim of the next tile is issued as the
-// current one starts, its record fetched two K slices into the current tile's
-// loads and published two slices later, so neither latency sits between two
-// tiles and the peer CTA's producer knows its next tile before it gets there.  A tile that
-// waits on earlier tiles therefore only ever waits on tiles that running pairs
-// have claimed: the launch makes progress however many of its pairs are
-// resident (other kernels may hold SMs), and the dynamic order also balances
-// tiles of unequal K across pairs.
+// Tiles are claimed, in list order, from a global ticket by a scheduler warp
+// of the leader CTA, which publishes each claimed tile's 32-byte record to
+// every role of both CTAs through a short ring in shared memory.  The ring's
+// depth bounds how far the scheduler runs ahead of the slowest role, so a
+// pair holds only the next few tiles; the claims and record fetches never
+// stall the producers, which only read the ring.  A tile that waits on
+// earlier tiles only ever waits on tiles that running pairs have claimed:
+// the launch makes progress however many of its pairs are resident (other
+// kernels may hold SMs), and the dynamic order also balances tiles of
+// unequal K across pairs.
 //
 // Every wait is bounded: on expiry the kernel records a timeout in the device
 // status word, drains its own copies and MMAs, frees TMEM and exits.
@@ -66,15 +67,17 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
 constexpr int EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int SCHED_WARP = 2 + EPI_WARPS;       // the tile scheduler (after the epilogue warps)
+constexpr int NUM_THREADS = 96 + 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;  // 2 accumulators x 256 fp32 columns
 constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
 constexpr int STORE_BOX_BYTES = 64 * 32;  // one TMA store box: 32 rows of 64 bytes
 constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per epilogue warp
-constexpr int SCHED = 8;  // depth of the tile-record ring
-// readers of every ring slot: the leader's MMA thread, the peer's producer,
-// and the epilogue warps of both CTAs
-constexpr uint32_t SCHED_READERS = 2 + 2 * EPI_WARPS;
+constexpr int SCHED = 4;  // depth of the tile-record ring: the scheduler's lookahead
+// readers of every ring slot: in the leader its producer, its MMA thread and
+// its epilogue warps; in the peer its producer and its epilogue warps
+constexpr uint32_t SCHED_READERS_LEADER = 2 + EPI_WARPS;
+constexpr uint32_t SCHED_READERS_PEER = 1 + EPI_WARPS;
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 1024 /*barriers, ring*/;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
 
@@ -86,13 +89,14 @@ struct RingRec {
 constexpr unsigned kRingEnd = 0xFFFFFFFFu;
 
 struct Shared {
-    RingRec ring[SCHED];     // claimed tiles' records (leader's producer writes both CTAs')
+    RingRec ring[SCHED];     // claimed tiles' records (the scheduler writes both CTAs')
     uint64_t full[STAGES];   // leader: both CTAs' operand bytes landed
     uint64_t empty[STAGES];  // each CTA: its slot may be refilled (leader's MMA commit)
     uint64_t tfull[2];       // each CTA: accumulator ready (leader's MMA commit)
     uint64_t tempty[2];      // leader: all 2 x EPI_WARPS epilogue warps drained the accumulator
-    uint64_t sfull[SCHED];   // each CTA: ring slot holds a record (leader's producer)
-    uint64_t sempty[SCHED];  // leader: every reader of both CTAs has read the ring slot
+    uint64_t sfull[SCHED];     // each CTA: ring slot holds a record (leader's producer)
+    uint64_t sempty_l[SCHED];  // leader: the leader's readers have read the slot (CTA scope)
+    uint64_t sempty_p[SCHED];  // leader: the peer's readers have read the slot (cluster scope)
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -130,21 +134,24 @@ __device__ __forceinline__ void record_timeout(Shared* sh, DeviceStatus* st) {
     *reinterpret_cast<volatile int*>(&sh->abort) = 1;
 }
 
-// Writer side of the tile ring (the leader's producer): publish a record in
+// Writer side of the tile ring (the leader's scheduler warp): publish a record in
 // the same slot of both CTAs' rings once every reader has read that slot's
-// previous record.  False when that wait ran out.
+// previous record.  The leader CTA's own readers synchronise with it at CTA
+// scope (plain shared-memory stores, CTA-scope release and acquire); only
+// the link to the peer CTA uses cluster scope.  False when a wait ran out.
 struct RingWriter {
     int slot = 0;
     uint32_t phase = 0;
     __device__ bool push(Shared* sh, const RingRec& rec, volatile int* abort_flag, unsigned long long limit) {
-        if (!mbar_wait_cluster(&sh->sempty[slot], phase ^ 1u, abort_flag, limit)) return false;
-        const uint32_t v = smem_u32(&sh->ring[slot]), b = smem_u32(&sh->sfull[slot]);
-#pragma unroll
-        for (uint32_t r = 0; r < 2; ++r) {
-            st_shared_cluster_v4(map_to_cta(v, r), rec.a);
-            st_shared_cluster_v4(map_to_cta(v + 16, r), rec.b);
-            mbar_arrive_cluster(map_to_cta(b, r));  // release: the record is visible first
-        }
+        if (!mbar_wait(&sh->sempty_l[slot], phase ^ 1u, abort_flag, limit)) return false;
+        if (!mbar_wait_cluster(&sh->sempty_p[slot], phase ^ 1u, abort_flag, limit)) return false;
+        st_shared_v4(smem_u32(&sh->ring[slot]), rec.a);
+        st_shared_v4(smem_u32(&sh->ring[slot]) + 16, rec.b);
+        mbar_arrive(&sh->sfull[slot]);  // release (CTA scope): the record is visible first
+        const uint32_t v = map_to_cta(smem_u32(&sh->ring[slot]), 1);
+        st_shared_cluster_v4(v, rec.a);
+        st_shared_cluster_v4(v + 16, rec.b);
+        mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sfull[slot]), 1));  // release (cluster scope)
         if (++slot == SCHED) {
             slot = 0;
             phase ^= 1u;
@@ -154,15 +161,21 @@ struct RingWriter {
 };
 
 // Reader side: the next published record (false when the wait ran out).
+// `leader`: this reader runs in the leader CTA (CTA-scope synchronisation).
 struct RingReader {
     int slot = 0;
     uint32_t phase = 0;
-    __device__ bool pop(Shared* sh, RingRec& rec, volatile int* abort_flag, unsigned long long limit) {
-        if (!mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit)) return false;
+    __device__ bool pop(Shared* sh, RingRec& rec, bool leader, volatile int* abort_flag, unsigned long long limit) {
+        const bool got = leader ? mbar_wait(&sh->sfull[slot], phase, abort_flag, limit)
+                                : mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit);
+        if (!got) return false;
         const volatile uint4* p = reinterpret_cast<const volatile uint4*>(&sh->ring[slot]);
         rec.a = make_uint4(p[0].x, p[0].y, p[0].z, p[0].w);
         rec.b = make_uint4(p[1].x, p[1].y, p[1].z, p[1].w);
-        mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sempty[slot]), 0));  // read: the slot is free
+        if (leader)
+            mbar_arrive(&sh->sempty_l[slot]);  // read: the slot is free (CTA scope)
+        else
+            mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sempty_p[slot]), 0));
         if (++slot == SCHED) {
             slot = 0;
             phase ^= 1u;
@@ -171,8 +184,9 @@ struct RingReader {
     }
     // The next record if it is already published, without consuming it (its
     // slot cannot be rewritten before this reader has popped it).
-    __device__ bool peek(Shared* sh, RingRec& rec) {
-        if (!mbar_try_wait_cluster(&sh->sfull[slot], phase)) return false;
+    __device__ bool peek(Shared* sh, RingRec& rec, bool leader) {
+        if (!(leader ? mbar_try_wait(&sh->sfull[slot], phase) : mbar_try_wait_cluster(&sh->sfull[slot], phase)))
+            return false;
         const volatile uint4* p = reinterpret_cast<const volatile uint4*>(&sh->ring[slot]);
         rec.a = make_uint4(p[0].x, p[0].y, p[0].z, p[0].w);
         rec.b = make_uint4(p[1].x, p[1].y, p[1].z, p[1].w);
@@ -192,33 +206,21 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     bool ok = true;
     int last_a = -1, last_b = -1;
     unsigned seen_mat = ~0u, seen_done = 0;  // counters only grow within a launch
-    RingWriter wr;
     RingReader rd;
-    // The leader claims tiles and publishes their records to both CTAs'
-    // rings one tile ahead; the peer reads them.  The claim of the next tile
-    // is issued when the current one starts and consumed two K slices into
-    // its loads, where the next record is fetched; it is published two slices
-    // later.  The next tile's dependency and tensor maps are acquired right
-    // after the current tile's last fill is issued (the slices still queued
-    // hide the wait).
+    // Both producers read the tile ring (the scheduler warp claims and
+    // publishes ahead).  The next tile's dependency and tensor maps are
+    // acquired right after the current tile's last fill is issued (the
+    // slices still queued hide the wait).
     bool early = false;  // the current tile's dependency was acquired early
-    RingRec cur;
-    if (leader) {
-        const unsigned t0 = atomicAdd(L.ticket, 1u);
-        cur = t0 < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(t0)) : end_rec();
-        if (!wr.push(sh, cur, abort_flag, lim)) ok = false;
-    }
     while (ok) {
-        if (!leader && !rd.pop(sh, cur, abort_flag, lim)) {
+        RingRec cur;
+        if (!rd.pop(sh, cur, leader, abort_flag, lim)) {
             ok = false;
             break;
         }
         if (cur.a.x == kRingEnd) break;
         const TcTile tile = decode_tile(cur);
-        unsigned claim = 0;
-        if (leader) claim = atomicAdd(L.ticket, 1u);
         RingRec nxt_rec;
-        bool have_next = false, pushed = false;
         // operands produced by earlier chain slots of the same matrix
         if (tile.need && !(tile.mat == seen_mat && tile.need <= seen_done)) {
             if (!early && !wait_counter(L.done + tile.mat, tile.need, abort_flag, lim)) {
@@ -284,21 +286,9 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 stage = 0;
                 phase ^= 1u;
             }
-            if (leader && !have_next && (kb >= 2 || kb == nk - 1)) {
-                nxt_rec = claim < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(claim))
-                                                                  : end_rec();
-                have_next = true;
-            }
-            if (leader && have_next && !pushed && (kb >= 4 || kb == nk - 1)) {
-                if (!wr.push(sh, nxt_rec, abort_flag, lim)) {
-                    ok = false;
-                    break;
-                }
-                pushed = true;
-            }
         }
-        if (ok && !leader) have_next = rd.peek(sh, nxt_rec);  // published already?
-        if (ok && have_next && nxt_rec.a.x != kRingEnd) {
+        // the next tile, if the scheduler has published it already
+        if (ok && rd.peek(sh, nxt_rec, leader) && nxt_rec.a.x != kRingEnd) {
             const TcTile nxt = decode_tile(nxt_rec);
             if (nxt.need && !(nxt.mat == seen_mat && nxt.need <= seen_done))
                 early = ld_acquire_gpu(L.done + nxt.mat) >= nxt.need;
@@ -314,7 +304,6 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 last_b = nxt.b_map;
             }
         }
-        if (leader) cur = nxt_rec;  // pushed in the K loop (ok) or not needed (timed out)
     }
     if (!ok) record_timeout(sh, L.status);
     // Drain (leader): the last fills of every stage must have landed before
@@ -331,6 +320,24 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     }
 }
 
+// The tile scheduler (one thread of the leader CTA): claims tiles in list
+// order and publishes their records until the list is exhausted, then the end
+// marker.  Its waits are only for free ring slots.
+__device__ void scheduler(const TcLaunch& L, Shared* sh) {
+    volatile int* abort_flag = &sh->abort;
+    const unsigned long long lim = L.wait_ns;
+    RingWriter wr;
+    while (true) {
+        const unsigned t = atomicAdd(L.ticket, 1u);
+        const RingRec rec = t < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(t)) : end_rec();
+        if (!wr.push(sh, rec, abort_flag, lim)) {
+            record_timeout(sh, L.status);
+            return;
+        }
+        if (rec.a.x == kRingEnd) return;
+    }
+}
+
 __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base) {
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
@@ -344,7 +351,7 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     RingReader rd;
     while (ok) {
         RingRec rec;
-        if (!rd.pop(sh, rec, abort_flag, lim)) {  // published as the producer starts its loads
+        if (!rd.pop(sh, rec, true, abort_flag, lim)) {  // the MMA thread runs in the leader CTA
             ok = false;
             break;
         }
@@ -432,7 +439,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     while (true) {
         RingRec rec;
         int got_rec = 1;
-        if (lane == 0) got_rec = rd.pop(sh, rec, abort_flag, lim) ? 1 : 0;
+        if (lane == 0) got_rec = rd.pop(sh, rec, rank == 0, abort_flag, lim) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, got_rec, 0)) {
             timed_out = true;
             break;
@@ -597,8 +604,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             mbar_init(&sh->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
         }
         for (int r = 0; r < SCHED; ++r) {
-            mbar_init(&sh->sfull[r], 1);              // the leader's producer publishes
-            mbar_init(&sh->sempty[r], SCHED_READERS);  // used in the leader only
+            mbar_init(&sh->sfull[r], 1);                       // the scheduler publishes
+            mbar_init(&sh->sempty_l[r], SCHED_READERS_LEADER);  // used in the leader only
+            mbar_init(&sh->sempty_p[r], SCHED_READERS_PEER);    // used in the leader only
         }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
@@ -618,6 +626,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) producer(L, tiles_smem, sh, rank);
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base);
+    } else if (warp == SCHED_WARP) {
+        if (lane == 0 && rank == 0) scheduler(L, sh);
     } else {
         epilogue_warps(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank);
     }

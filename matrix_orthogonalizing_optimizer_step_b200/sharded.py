@@ -65,8 +65,15 @@ def loads(shapes, owner, world_size, steps=5):
 _GATHER_BUFS = {}
 
 
+def release_gather_buffers():
+    """Drop the flat buffers that gather_owned keeps between steps (one per
+    dtype and device, as large as the padded all-gather of that dtype)."""
+    _GATHER_BUFS.clear()
+
+
 def _gather_buffer(numel, dtype, device):
-    """A cached flat buffer of at least numel elements (reused across steps)."""
+    """A cached flat buffer of at least numel elements (reused across steps;
+    release_gather_buffers frees them)."""
     key = (dtype, str(device))
     buf = _GATHER_BUFS.get(key)
     if buf is None or buf.numel() < numel:

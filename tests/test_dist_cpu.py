@@ -89,6 +89,9 @@ def _worker(rank, world, port, out_q):
         import bench
         mx = bench.max_over_ranks(float(rank + 1) * 1.5, world)
         bench.barrier(world)
+        assert sharded._GATHER_BUFS  # kept for the next step ...
+        sharded.release_gather_buffers()
+        assert not sharded._GATHER_BUFS  # ... until released
         out_q.put((rank, owner, [p.numpy().copy() for p in P], [m.float().numpy().copy() for m in M], mx))
     finally:
         dist.destroy_process_group()

@@ -126,3 +126,42 @@ def test_hybrid_argument_error_enqueues_nothing():
     torch.cuda.synchronize()
     assert mo.muon_launch_count() == n0
     assert all(torch.equal(a, b) for a, b in zip(W, W0))
+
+
+@pytest.mark.parametrize("grad_dt,par_dt,mom_dt,lam", [
+    ("bf16", "f32", "bf16", 0.0), ("f32", "f32", "bf16", 0.0), ("bf16", "bf16", "bf16", 0.0),
+    ("bf16", "f32", "f32", 0.0), ("f32", "bf16", "f32", 0.0), ("bf16", "f32", "bf16", 0.06),
+    ("f32", "f32", "f32", 0.06)])
+def test_hybrid_instances_equal_separate_calls(grad_dt, par_dt, mom_dt, lam):
+    """Every instance of the hybrid momentum launch (gradient dtype x momentum
+    dtype x soft-threshold split, with fp32 or bf16 parameters) gives the
+    same bits as muon_step followed by muon_adamw_step."""
+    code = {"f32": mo.MUON_DTYPE_F32, "bf16": mo.MUON_DTYPE_BF16}
+    mo.muon_reset_config()
+    mo.muon_set_config(grad_dtype=code[grad_dt], param_dtype=code[par_dt], momentum_dtype=code[mom_dt],
+                       soft_threshold=lam)
+    shapes = [(256, 768), (768, 256), (200, 712), (37, 91)]
+    numels = [1024 * 768, 768, 2304, 5, 4099]
+
+    def lanes():
+        G = [wl.make_single(r, c, 4300 + i, "student_t3_outl", DEV, grad_dt, 0.01) for i, (r, c) in enumerate(shapes)]
+        M = [wl.make_single(r, c, 4400 + i, "student_t3", DEV, mom_dt, 0.01) for i, (r, c) in enumerate(shapes)]
+        W = [wl.make_single(r, c, 4500 + i, "params", DEV, par_dt) for i, (r, c) in enumerate(shapes)]
+        P = [wl.make_single(1, n, 4600 + i, "params", DEV, par_dt).view(-1) for i, n in enumerate(numels)]
+        AG = [wl.make_single(1, n, 4700 + i, "student_t3", DEV, grad_dt, 0.01).view(-1) for i, n in enumerate(numels)]
+        M1 = [torch.zeros(n, device=DEV) for n in numels]
+        M2 = [torch.zeros(n, device=DEV) for n in numels]
+        return W, G, M, P, AG, M1, M2
+
+    W, G, M, P, AG, M1, M2 = lanes()
+    Wb, _, Mb, Pb, _, M1b, M2b = lanes()
+    for t in (1, 2):
+        mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, t, lr=0.02, adam_lr=1e-3)
+        mo.muon_step(Wb, G, Mb, mu=0.95, nesterov=True, lr=0.02)
+        mo.muon_adamw_step(Pb, AG, M1b, M2b, t, lr=1e-3)
+    torch.cuda.synchronize()
+    for x, y in zip(W + M + P + M1 + M2, Wb + Mb + Pb + M1b + M2b):
+        assert torch.equal(x, y)
+    st, _ = mo.muon_device_status()
+    assert st == mo.MUON_OK
+    mo.muon_reset_config()

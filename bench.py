@@ -446,6 +446,54 @@ def measure_extra(w, dev, args, peaks, peak_src, world):
     return out
 
 
+def time_hybrid_lane(w, dev, steps, peaks, world):
+    """The hybrid step's elementwise launch (muon_hybrid_step: the Muon
+    momentum pass with the model's AdamW parameters appended to its grid),
+    from the library's per-launch events: GB/s of the combined launch against
+    the measured HBM copy bandwidth, next to the two lanes timed as separate
+    launches (muon_step's momentum launch, muon_adamw_step)."""
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+    mo.muon_reset_config()
+    W = [wl.make_matrix(w, i, wl.ROLE_PARAM, device=dev) for i in range(w.count)]
+    G = [wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev) for i in range(w.count)]
+    M = [wl.make_matrix(w, i, wl.ROLE_MOMENTUM, device=dev) for i in range(w.count)]
+    numels = list(w.adamw_numels)
+    P = [wl.make_single(1, n, 5000 + i, "params", dev, "f32").view(-1) for i, n in enumerate(numels)]
+    AG = [wl.make_single(1, n, 6000 + i, "student_t3", dev, "bf16", 0.01).view(-1) for i, n in enumerate(numels)]
+    M1 = [torch.zeros(n, device=dev) for n in numels]
+    M2 = [torch.zeros(n, device=dev) for n in numels]
+
+    def measure(fn):
+        for t in range(1, 4):
+            fn(t)
+        torch.cuda.synchronize()
+        mo.muon_profile_reset()
+        mo.muon_profile_enable(True)
+        for t in range(4, 4 + steps):
+            fn(t)
+        prof = mo.muon_profile_read()
+        mo.muon_profile_enable(False)
+        return prof
+
+    hyb = measure(lambda t: mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, t))
+    sep = measure(lambda t: (mo.muon_step(W, G, M), mo.muon_adamw_step(P, AG, M1, M2, t)))
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    k = hyb["momentum_norm"]
+    gbs = k["bytes"] / (k["total_ms"] * 1e-3) / 1e9
+    sep_ms = (sep["momentum_norm"]["total_ms"] + sep["adamw"]["total_ms"]) / steps
+    out = {"kernel": "momentum_norm, hybrid instance (Muon momentum pass + AdamW lane, one launch)",
+           "workload": w.name, "muon_elements": w.elements, "adamw_elements": sum(numels),
+           "ms": round(k["total_ms"] / steps, 4), "bound": "hbm", "achieved": round(gbs, 1), "peak": peak,
+           "unit": "GB/s", "frac": round(gbs / peak, 4) if peak else None,
+           "separate_launches_ms": round(sep_ms, 4), "launches_per_step": k["launches"] / steps}
+    mo.muon_reset_config()
+    del W, G, M, P, AG, M1, M2
+    torch.cuda.empty_cache()
+    mo.muon_release_workspace()
+    return out
+
+
 def run_ours(args):
     import torch
     import matrix_orthogonalizing_optimizer_step_b200 as mo
@@ -563,6 +611,11 @@ def run_ours(args):
     if w.adamw_numels and not args.no_adamw:
         adamw = time_adamw_lane(w, dev, max(args.steps, 5), peaks, world)
 
+    # ---- the hybrid step's single elementwise launch (GPT-2 124M set) --------
+    hybrid = None
+    if world == 1 and not args.no_adamw:
+        hybrid = time_hybrid_lane(wl.WORKLOADS[2], dev, max(args.steps, 5), peaks, world)
+
     # ---- other workloads, device-timed (extra keys) ----------------------------
     extra = {}
     also = [int(x) for x in args.also.split(",") if x.strip() and int(x) != w.wid] if world == 1 else []
@@ -597,6 +650,7 @@ def run_ours(args):
             "gpu_launches": int(launches),
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
             "adamw_lane": adamw,
+            "hybrid_lane": hybrid,
             "also": extra,
         }
         print(json.dumps(out), flush=True)

@@ -12,7 +12,7 @@ constexpr int kThreads = 256;
 
 template <bool P_F32, bool G_F32>
 __global__ void __launch_bounds__(kThreads) adamw_kernel(const AdamLaunch L) {
-    adamw_chunk<P_F32, G_F32>(L, blockIdx.x);
+    adamw_chunk<P_F32, G_F32, 8>(L, blockIdx.x);
 }
 
 }  // namespace

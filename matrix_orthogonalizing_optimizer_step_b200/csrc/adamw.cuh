@@ -44,49 +44,73 @@ __device__ __forceinline__ float adam_elem(float p, float g, float& m, float& v,
     return p - k.lr_c1 * m / (sqrtf(v * k.c2) + k.eps);
 }
 
-// AdamW on chunk `chunk` of the launch's tensors, by the whole CTA (blockDim.x threads).
-template <bool P_F32, bool G_F32>
+// AdamW on chunk `chunk` of the launch's tensors, by the whole CTA (blockDim.x
+// threads).  VEC elements per thread and iteration when the tensor is aligned:
+// 8 (two 16-byte accesses per fp32 array, one per 16-bit array) in the AdamW
+// launch; 4 in the hybrid launch, where the AdamW body shares a kernel with
+// the momentum pass and must not raise its register count (and lower its
+// occupancy) much.
+template <bool P_F32, bool G_F32, int VEC>
 __device__ __forceinline__ void adamw_chunk(const AdamLaunch& L, long long chunk) {
+    static_assert(VEC == 4 || VEC == 8, "vector width");
     const AdamTensor T = L.tensors[adam_find_tensor(L.tensors, L.ntensors, chunk)];
     const long long e0 = (chunk - T.chunk_begin) * kMomChunk;
     const AdamCoef k{L.decay, L.beta1, 1.f - L.beta1, L.beta2, 1.f - L.beta2, L.lr_c1, L.c2, L.eps};
     const int pdt = P_F32 ? DT_F32 : DT_BF16;
     const int nthr = static_cast<int>(blockDim.x);
-    if (T.vec_ok) {
-        // 8 elements per thread and iteration: two 16-byte accesses per fp32
-        // array, one per 16-bit array
-        for (int i = threadIdx.x; i < kMomChunk / 8; i += nthr) {
-            const long long e = e0 + 8LL * i;
+    if (T.vec_ok) {  // numel % 8 == 0, every pointer 16-byte aligned
+        for (int i = threadIdx.x; i < kMomChunk / VEC; i += nthr) {
+            const long long e = e0 + static_cast<long long>(VEC) * i;
             if (e >= T.numel) break;
-            float p[8], g[8], m[8], v[8];
-            auto ld8f = [](const float* src, float* dst) {
-                const float4 a = *reinterpret_cast<const float4*>(src);
-                const float4 b = *reinterpret_cast<const float4*>(src + 4);
-                dst[0] = a.x, dst[1] = a.y, dst[2] = a.z, dst[3] = a.w;
-                dst[4] = b.x, dst[5] = b.y, dst[6] = b.z, dst[7] = b.w;
-            };
-            auto st8f = [](float* dst, const float* src) {
-                *reinterpret_cast<float4*>(dst) = make_float4(src[0], src[1], src[2], src[3]);
-                *reinterpret_cast<float4*>(dst + 4) = make_float4(src[4], src[5], src[6], src[7]);
-            };
-            if (P_F32)
-                ld8f(static_cast<const float*>(T.p) + e, p);
-            else
-                unpack8(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(T.p) + e), DT_BF16, p);
-            if (G_F32)
-                ld8f(static_cast<const float*>(T.g) + e, g);
-            else
-                unpack8(*reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(T.g) + e), DT_BF16, g);
-            ld8f(T.m + e, m);
-            ld8f(T.v + e, v);
+            float p[VEC], g[VEC], m[VEC], v[VEC];
+            auto ldf = [](const float* src, float* dst) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) p[j] = adam_elem(p[j], g[j], m[j], v[j], k);
-            st8f(T.m + e, m);
-            st8f(T.v + e, v);
+                for (int q = 0; q < VEC / 4; ++q) {
+                    const float4 a = *reinterpret_cast<const float4*>(src + 4 * q);
+                    dst[4 * q] = a.x, dst[4 * q + 1] = a.y, dst[4 * q + 2] = a.z, dst[4 * q + 3] = a.w;
+                }
+            };
+            auto stf = [](float* dst, const float* src) {
+#pragma unroll
+                for (int q = 0; q < VEC / 4; ++q)
+                    *reinterpret_cast<float4*>(dst + 4 * q) =
+                        make_float4(src[4 * q], src[4 * q + 1], src[4 * q + 2], src[4 * q + 3]);
+            };
+            // VEC bf16 values: one 16-byte access (8) or one 8-byte access (4)
+            auto ld16 = [](const void* base, long long off, float* dst) {
+                const uint16_t* q = static_cast<const uint16_t*>(base) + off;
+                if (VEC == 8) {
+                    unpack8(*reinterpret_cast<const uint4*>(q), DT_BF16, dst);
+                } else {
+                    const uint2 w = *reinterpret_cast<const uint2*>(q);
+                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+                    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+                    dst[0] = a.x, dst[1] = a.y, dst[2] = b.x, dst[3] = b.y;
+                }
+            };
             if (P_F32)
-                st8f(static_cast<float*>(T.p) + e, p);
+                ldf(static_cast<const float*>(T.p) + e, p);
             else
+                ld16(T.p, e, p);
+            if (G_F32)
+                ldf(static_cast<const float*>(T.g) + e, g);
+            else
+                ld16(T.g, e, g);
+            ldf(T.m + e, m);
+            ldf(T.v + e, v);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) p[j] = adam_elem(p[j], g[j], m[j], v[j], k);
+            stf(T.m + e, m);
+            stf(T.v + e, v);
+            if (P_F32) {
+                stf(static_cast<float*>(T.p) + e, p);
+            } else if (VEC == 8) {
                 *reinterpret_cast<uint4*>(static_cast<uint16_t*>(T.p) + e) = pack8(p, DT_BF16);
+            } else {
+                __nv_bfloat162 a = __floats2bfloat162_rn(p[0], p[1]), b = __floats2bfloat162_rn(p[2], p[3]);
+                *reinterpret_cast<uint2*>(static_cast<uint16_t*>(T.p) + e) =
+                    make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+            }
         }
     } else {
         for (int i = threadIdx.x; i < kMomChunk; i += nthr) {

@@ -93,9 +93,9 @@ __global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch
     if (HYBRID && chunk >= L.nchunks) {
         // hybrid step: the AdamW lane's chunks follow the Muon chunks
         if (L.adam.p_dt == DT_F32)
-            adamw_chunk<true, G_F32>(L.adam, chunk - L.nchunks);
+            adamw_chunk<true, G_F32, 4>(L.adam, chunk - L.nchunks);
         else
-            adamw_chunk<false, G_F32>(L.adam, chunk - L.nchunks);
+            adamw_chunk<false, G_F32, 4>(L.adam, chunk - L.nchunks);
         return;
     }
     if (chunk == 0 && L.done)  // the GEMM launches that follow count completions and tickets from zero

@@ -17,11 +17,20 @@
 //               the transaction bytes of both CTAs land on the leader's barrier
 //   warp 1      TMEM owner (both CTAs) and MMA issuer (leader only):
 //               two 256-column fp32 accumulators (double-buffered)
-//   warps 2..9  epilogue: tcgen05.ld of 32-column slices, fused combine
+//   warps 2..9  epilogue: tcgen05.ld of 32-column slices of the warp's TMEM
+//               lane quarter (32 rows), fused combine
 //               sigma*(alpha*acc + beta*C1) + gamma*C2 + delta*I; each warp
-//               stages its 32 x 32 result in a 64-byte-swizzled box in
-//               shared memory and one lane stores it with a TMA bulk store
-//               (outputs with an unaligned row pitch: direct stores)
+//               stages its 32 x 32 result in a 64-byte-swizzled box in shared
+//               memory and one lane stores it with a TMA bulk store (outputs
+//               with an unaligned row pitch: direct stores).  Persistent
+//               launches run them as one group: all eight warps take every
+//               tile (two per lane quarter, 128 columns each).  Chained
+//               launches (short K, one chain counter per tile) run them as
+//               two groups of four, one per accumulator: group g takes the
+//               pair's tiles g, g + 2, g + 4, ... (all 256 columns), so the
+//               fixed per-tile latencies of one group (tile record, problem,
+//               dependency, store completion, chain counter) overlap the
+//               other group's work.
 //
 // Symmetric outputs (X X^T and every product of polynomials in R) are only
 // computed and stored for the upper 256 x 256 tiles; consumers read a lower
@@ -47,6 +56,8 @@
 //
 // Every wait is bounded: on expiry the kernel records a timeout in the device
 // status word, drains its own copies and MMAs, frees TMEM and exits.
+#include <algorithm>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -74,10 +85,23 @@ constexpr int MN_BLOCK_BYTES = 64 * BK * 2;  // one 64 (MN) x 64 (K) box
 constexpr int STORE_BOX_BYTES = 64 * 32;  // one TMA store box: 32 rows of 64 bytes
 constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per epilogue warp
 constexpr int SCHED = 4;  // depth of the tile-record ring: the scheduler's lookahead
-// readers of every ring slot: in the leader its producer, its MMA thread and
-// its epilogue warps; in the peer its producer and its epilogue warps
-constexpr uint32_t SCHED_READERS_LEADER = 2 + EPI_WARPS;
-constexpr uint32_t SCHED_READERS_PEER = 1 + EPI_WARPS;
+// The epilogue warps as GROUPS groups (1 or 2), each taking every GROUPS-th
+// tile of the pair.
+template <int GROUPS>
+struct EpiShape {
+    static constexpr int group_warps = EPI_WARPS / GROUPS;
+    static constexpr int cols = BN / (group_warps / 4);  // tile columns per epilogue warp
+    // readers of every ring slot: in the leader its producer, its MMA thread
+    // and the epilogue warps of the group that takes the tile; in the peer
+    // its producer and that group's epilogue warps
+    static constexpr uint32_t readers_leader = 2 + group_warps;
+    static constexpr uint32_t readers_peer = 1 + group_warps;
+    static_assert(group_warps % 4 == 0, "a group covers the four TMEM lane quarters");
+    static_assert(2 % GROUPS == 0 && SCHED % GROUPS == 0, "a group owns whole accumulators and ring slots");
+};
+constexpr int kChainGroups = 2;  // epilogue groups of a chained launch (persistent launches: 1)
+static_assert(kTileArrivals == 2 * EpiShape<kChainGroups>::group_warps,
+              "chain completions are counted per tile: one group's warps in each CTA");
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 1024 /*barriers, ring*/;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
 
@@ -93,7 +117,7 @@ struct Shared {
     uint64_t full[STAGES];   // leader: both CTAs' operand bytes landed
     uint64_t empty[STAGES];  // each CTA: its slot may be refilled (leader's MMA commit)
     uint64_t tfull[2];       // each CTA: accumulator ready (leader's MMA commit)
-    uint64_t tempty[2];      // leader: all 2 x EPI_WARPS epilogue warps drained the accumulator
+    uint64_t tempty[2];      // leader: the owning group's warps of both CTAs drained the accumulator
     uint64_t sfull[SCHED];     // each CTA: ring slot holds a record (leader's producer)
     uint64_t sempty_l[SCHED];  // leader: the leader's readers have read the slot (CTA scope)
     uint64_t sempty_p[SCHED];  // leader: the peer's readers have read the slot (cluster scope)
@@ -162,9 +186,12 @@ struct RingWriter {
 
 // Reader side: the next published record (false when the wait ran out).
 // `leader`: this reader runs in the leader CTA (CTA-scope synchronisation).
+// An epilogue group reads every GROUPS-th record, from slot `first` on.
 struct RingReader {
     int slot = 0;
     uint32_t phase = 0;
+    int stride = 1;
+    __device__ RingReader(int first = 0, int step = 1) : slot(first), stride(step) {}
     __device__ bool pop(Shared* sh, RingRec& rec, bool leader, volatile int* abort_flag, unsigned long long limit) {
         const bool got = leader ? mbar_wait(&sh->sfull[slot], phase, abort_flag, limit)
                                 : mbar_wait_cluster(&sh->sfull[slot], phase, abort_flag, limit);
@@ -176,8 +203,9 @@ struct RingReader {
             mbar_arrive(&sh->sempty_l[slot]);  // read: the slot is free (CTA scope)
         else
             mbar_arrive_cluster(map_to_cta(smem_u32(&sh->sempty_p[slot]), 0));
-        if (++slot == SCHED) {
-            slot = 0;
+        slot += stride;
+        if (slot >= SCHED) {
+            slot -= SCHED;
             phase ^= 1u;
         }
         return true;
@@ -321,20 +349,24 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
 }
 
 // The tile scheduler (one thread of the leader CTA): claims tiles in list
-// order and publishes their records until the list is exhausted, then the end
-// marker.  Its waits are only for free ring slots.
+// order and publishes their records until the list is exhausted, then one end
+// marker per epilogue group (the producers and the MMA thread stop at the
+// first).  Its waits are only for free ring slots.
+template <int GROUPS>
 __device__ void scheduler(const TcLaunch& L, Shared* sh) {
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
     RingWriter wr;
-    while (true) {
-        const unsigned t = atomicAdd(L.ticket, 1u);
+    int ends = 0;
+    while (ends < GROUPS) {
+        unsigned t = static_cast<unsigned>(L.ntiles);
+        if (ends == 0) t = atomicAdd(L.ticket, 1u);
         const RingRec rec = t < static_cast<unsigned>(L.ntiles) ? load_tile_raw(L.tiles, static_cast<int>(t)) : end_rec();
         if (!wr.push(sh, rec, abort_flag, lim)) {
             record_timeout(sh, L.status);
             return;
         }
-        if (rec.a.x == kRingEnd) return;
+        if (rec.a.x == kRingEnd) ++ends;
     }
 }
 
@@ -416,15 +448,19 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     }
 }
 
+template <int GROUPS>
 __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint32_t tmem_base, int warp, int lane,
                                uint32_t rank) {
+    using S = EpiShape<GROUPS>;
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
-    const int q = warp & 3;            // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;  // column half of the tile
+    const int q = warp & 3;                       // TMEM lane quarter this warp may access
+    const int group = (warp - 2) / S::group_warps;       // takes the pair's tiles group, group + GROUPS, ...
+    const int part = ((warp - 2) % S::group_warps) >> 2;  // column part of the tile
     const uint32_t tempty_leader[2] = {map_to_cta(smem_u32(&sh->tempty[0]), 0),
                                        map_to_cta(smem_u32(&sh->tempty[1]), 0)};
-    int acc = 0;
+    // tile i of the pair uses accumulator i % 2 (the MMA thread alternates)
+    int acc = group % 2;
     uint32_t acc_phase = 0;
     unsigned seen_mat = ~0u, seen_done = 0;
     uint32_t nstored = 0;  // TMA store boxes issued by this warp (alternating buffers)
@@ -434,7 +470,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     const uint32_t sw = (static_cast<uint32_t>(lane) >> 1) & 3u;
     // lane 0 reads the tile ring for the warp (one reader per warp) and
     // passes the record's first half (problem, position, matrix, dependency)
-    RingReader rd;
+    RingReader rd(group, GROUPS);
     bool timed_out = false;
     while (true) {
         RingRec rec;
@@ -467,7 +503,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         const float sig = ep.sigma ? *ep.sigma : 1.f;
         const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;  // this warp's first row
         const long long row = row0 + lane;
-        const int cbase = bj * BN + half * (BN / 2);
+        const int cbase = bj * BN + part * S::cols;
         const bool use_tma = ep.o1_map >= 0;
         const CUtensorMap* omap = use_tma ? L.maps + ep.o1_map : nullptr;
         if (use_tma && ep.o1_map != last_map) {
@@ -480,12 +516,12 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         Raw32 pre;
         prefetch_row32(ep, PM, PN, row, cbase, pre);
         // C2 (the parameters of the fused update, read once from DRAM): pull
-        // this lane's row of the warp's 128 columns into L2 now, so the
-        // per-slice loads below hit L2
+        // this lane's row of the warp's columns into L2 now, so the per-slice
+        // loads below hit L2
         if (ep.c2 && !skip && row < PM) {
             const int es = ep.c2_dt == DT_F32 ? 4 : 2;
             const char* p = static_cast<const char*>(ep.c2) + (row * ep.ldc2 + cbase) * es;
-            const int bytes = min(BN / 2, PN - cbase) * es;
+            const int bytes = min(S::cols, PN - cbase) * es;
             for (int o = 0; o < bytes; o += 128) prefetch_l2(p + o);
         }
         // every lane waits; the warp leaves together unless all lanes saw the
@@ -498,19 +534,18 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         tc_fence_after();
         // one slice per iteration, not unrolled: the epilogue's code stays small
 #pragma unroll 1
-        for (int c = 0; c < BN / 2; c += 32) {
+        for (int c = 0; c < S::cols; c += 32) {
             const int col0 = cbase + c;
             Raw32 nxt;  // C1 of the next slice, fetched while this one is processed
             nxt.ok = 0;
-            if (c + 32 < BN / 2) prefetch_row32(ep, PM, PN, row, col0 + 32, nxt);
+            if (c + 32 < S::cols) prefetch_row32(ep, PM, PN, row, col0 + 32, nxt);
             if (col0 >= PN) {  // warp-uniform
                 pre = nxt;
                 continue;
             }
             uint32_t r[32];
             __syncwarp();
-            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * (BN / 2) + c,
-                               r);
+            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + part * S::cols + c, r);
             tmem_wait_ld();
             if (skip || row0 >= PM) {  // warp-uniform
                 pre = nxt;
@@ -573,8 +608,9 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             __syncwarp();
             if (lane == 0) red_release_add_gpu(L.done + tile.mat, 1u);
         }
-        if (++acc == 2) {
-            acc = 0;
+        acc += GROUPS;  // this group's next tile
+        if (acc >= 2) {
+            acc -= 2;
             acc_phase ^= 1u;
         }
     }
@@ -584,8 +620,10 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     __syncwarp();
 }
 
+template <int GROUPS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ TcLaunch L) {
+    using S = EpiShape<GROUPS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem =
         reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -601,12 +639,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&sh->tfull[a], 1);
-            mbar_init(&sh->tempty[a], 2 * EPI_WARPS);  // every epilogue warp of both CTAs
+            mbar_init(&sh->tempty[a], 2 * S::group_warps);  // the owning group's warps of both CTAs
         }
         for (int r = 0; r < SCHED; ++r) {
             mbar_init(&sh->sfull[r], 1);                       // the scheduler publishes
-            mbar_init(&sh->sempty_l[r], SCHED_READERS_LEADER);  // used in the leader only
-            mbar_init(&sh->sempty_p[r], SCHED_READERS_PEER);    // used in the leader only
+            mbar_init(&sh->sempty_l[r], S::readers_leader);  // used in the leader only
+            mbar_init(&sh->sempty_p[r], S::readers_peer);    // used in the leader only
         }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
@@ -627,9 +665,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base);
     } else if (warp == SCHED_WARP) {
-        if (lane == 0 && rank == 0) scheduler(L, sh);
+        if (lane == 0 && rank == 0) scheduler<GROUPS>(L, sh);
     } else {
-        epilogue_warps(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank);
+        epilogue_warps<GROUPS>(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank);
     }
 
     tc_fence_before();
@@ -648,12 +686,12 @@ size_t gemm_tc_smem_bytes() { return SMEM_BYTES; }
 int gemm_tc_tile_m() { return BMP; }
 int gemm_tc_tile_n() { return BN; }
 
-// CTA pairs that can be resident at once (the chained launch needs all of its
-// pairs co-resident: a tile may wait for tiles of any other pair).
-int gemm_tc_max_pairs() {
-    static int cached = -1;
-    if (cached >= 0) return cached;
-    cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SMEM_BYTES));
+namespace {
+// CTA pairs of one instance that can be resident at once.
+template <int GROUPS>
+int max_pairs_of() {
+    cudaFuncSetAttribute(gemm_tc_kernel<GROUPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(SMEM_BYTES));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -666,24 +704,40 @@ int gemm_tc_max_pairs() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GROUPS>, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
-    cached = n;
     return n;
+}
+}  // namespace
+
+// CTA pairs that can be resident at once (either instance): the grid of a
+// persistent launch.
+int gemm_tc_max_pairs() {
+    static int cached = -1;
+    if (cached >= 0) return cached;
+    cached = std::min(max_pairs_of<1>(), max_pairs_of<kChainGroups>());
+    return cached;
 }
 
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream) {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(SMEM_BYTES));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_tc_kernel<kChainGroups>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(SMEM_BYTES));
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (L.ntiles <= 0) return cudaSuccess;
-    gemm_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(L);
+    // chained launches (chain counters) split the epilogue into two groups
+    if (L.done)
+        gemm_tc_kernel<kChainGroups><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(L);
+    else
+        gemm_tc_kernel<1><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(L);
     return cudaGetLastError();
 }
 

@@ -46,7 +46,7 @@ struct TcLaunch {
     DeviceStatus* status;
 };
 
-constexpr unsigned kTileArrivals = 16;  // epilogue warps of a CTA pair
+constexpr unsigned kTileArrivals = 8;  // epilogue warps of a CTA pair that take one tile (one group per CTA)
 
 size_t gemm_tc_smem_bytes();
 int gemm_tc_tile_m();

@@ -26,6 +26,12 @@ namespace muon {
 namespace {
 
 constexpr int kThreads = 256;
+// Eight resident CTAs per SM (every warp slot): at most 32 registers a
+// thread.  The momentum pass needs no more; the hybrid instance's AdamW body
+// would take 47-48 without the bound, and since registers are allocated per
+// kernel that would cost the momentum chunks of the same launch a third of
+// their occupancy (the bound costs the AdamW body a few spilled words instead).
+constexpr int kMinBlocks = 8;
 constexpr int kVecPerThread = kMomChunk / 8 / kThreads;  // 8-element vectors per thread
 static_assert(kVecPerThread * 8 * kThreads == kMomChunk, "chunk layout");
 
@@ -82,10 +88,10 @@ __device__ __forceinline__ T block_sum(T v, T* red) {
 }
 
 // HYBRID: the grid also carries the AdamW lane's chunks (after the Muon
-// chunks).  A separate instance, so that the plain Muon step keeps the small
-// register footprint (and the occupancy) of the momentum pass alone.
+// chunks).  A separate instance, so that the plain Muon step's code stays
+// that of the momentum pass alone.
 template <bool G_F32, int MOM, bool U_F32, bool CLIP, bool HYBRID>
-__global__ void __launch_bounds__(kThreads) momentum_norm_kernel(const MomLaunch L) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) momentum_norm_kernel(const MomLaunch L) {
     __shared__ float red_f[kThreads / 32];
     __shared__ double red_d[kThreads / 32];
     __shared__ int is_last;

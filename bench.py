@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--form", default="auto", choices=["auto", "standard", "gram"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--offload-chunks", type=int, default=8,
+                    help="groups of matrices the e2e leg's offload step pipelines its copies over")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-adamw", action="store_true",
                     help="skip the AdamW-lane measurement on the model's AdamW parameters")
@@ -564,19 +566,30 @@ def run_ours(args):
     if not args.no_e2e:
         e2e_steps = max(1, min(args.steps, 10))
         if w.full_step:
-            params, grads = inp["params"], inp["grads"]
+            params, grads, moms = inp["params"], inp["grads"], inp["moms"]
             host_g = [g.detach().to("cpu").pin_memory() for g in grads]
             host_p = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
+            # the offload step keeps one plan per group of matrices: free the
+            # whole-set plan of the device-timed step first
+            mo.muon_release_workspace()
+            if "owner" in inp:
+                from matrix_orthogonalizing_optimizer_step_b200 import sharded
 
-            def e2e_step():
-                for h, g in zip(host_g, grads):
-                    g.copy_(h, non_blocking=True)
-                step()
-                for h, p in zip(host_p, params):
-                    h.copy_(p, non_blocking=True)
+                def e2e_step():
+                    for h, g in zip(host_g, grads):
+                        g.copy_(h, non_blocking=True)
+                    sharded.sharded_step(params, grads, moms, mu=0.95, nesterov=True, lr=6e-4, owner=inp["owner"])
+                    for h, p in zip(host_p, params):
+                        h.copy_(p, non_blocking=True)
+                note = "pinned host grads -> HBM, sharded step, params -> pinned host, per step"
+            else:
+                def e2e_step():
+                    mo.muon_step_offload(params, grads, moms, grads_host=host_g, params_host=host_p,
+                                         mu=0.95, nesterov=True, lr=6e-4, chunks=args.offload_chunks)
+                note = (f"muon_step_offload: pinned host grads -> HBM and updated params -> pinned host, "
+                        f"pipelined with the step over {args.offload_chunks} groups of matrices, per step")
             h2d = inp["bytes_in"]
             d2h = sum(p.numel() * p.element_size() for p in params)
-            note = "pinned host grads -> HBM, muon_step, params -> pinned host, per step"
         else:
             work = inp["work"]
             host_in = {s: t.detach().to("cpu").pin_memory() for s, t in work.items()}
@@ -598,6 +611,7 @@ def run_ours(args):
         del e2e_step
         if w.full_step:
             del host_g, host_p
+            mo.muon_release_workspace()
         else:
             del host_in, host_out
 

@@ -232,6 +232,52 @@ MUON_API int muon_hybrid_step(void* const* params, const void* const* grads, voi
                               int nesterov, float lr, const int* shape_list, int count,
                               const muon_adamw_lane* adamw);
 
+/*
+ * muon_step_offload -- muon_step for a training loop that keeps gradients
+ * and/or the updated parameters in page-locked host memory, with the PCIe
+ * copies overlapped with the step.  The count matrices are split into
+ * min(chunks, count) groups of consecutive matrices with about equal copy
+ * bytes (the grouping of muon_offload_chunks).  All groups' gradients are
+ * copied in, in order, on a host-to-device copy stream; group k is stepped on
+ * the bound stream once its gradients have landed, and its updated
+ * parameters are copied out on a device-to-host copy stream as soon as its
+ * step has finished.  While group k is stepped, group k + 1's gradients come in and
+ * group k - 1's parameters go out, so both copy directions and the kernels
+ * run at once.
+ * params, grads, momentum, mu, nesterov, lr, shape_list, count: as muon_step
+ *               (grads are the device buffers the gradients are copied into)
+ * grads_host   host array of count page-locked host pointers (grad_dtype,
+ *               rows x cols row-major each), copied into grads; NULL: the
+ *               gradients are already in grads
+ * params_host  host array of count page-locked host pointers (param_dtype)
+ *               that receive the updated parameters; NULL: no copy out
+ * chunks       >= 1 (1: copy in, step, copy out, with no overlap)
+ * Each group is one muon_step with its own cached plan and workspace, so the
+ * results equal muon_step's bit for bit.  Host pointers that are not
+ * page-locked give MUON_ERR_INVALID_ARG (their copies could not overlap).
+ * Every argument is checked before anything is enqueued.  The call ends by
+ * making the bound stream wait for both copy streams: work enqueued on it
+ * afterwards, or a synchronize of it, comes after every copy.  A non-finite
+ * matrix is reported by muon_device_status in the caller's numbering.  If
+ * group k fails to run, groups before it are stepped and copied, later ones
+ * are not.  The copy streams and the per-group plans are the library's
+ * (muon_release_workspace frees the plans).
+ */
+MUON_API int muon_step_offload(void* const* params, const void* const* grads_host, void* const* grads,
+                               void* const* momentum, void* const* params_host, float mu, int nesterov, float lr,
+                               const int* shape_list, int count, int chunks);
+
+/*
+ * muon_offload_chunks -- the grouping of muon_step_offload: with bytes[i] >= 0
+ * the weight of matrix i, fills bounds (host int[g + 1]) with 0 = bounds[0] <
+ * bounds[1] < ... < bounds[g] = count: g = min(chunks, count) groups of
+ * consecutive matrices of about equal total weight.  Group k closes at the
+ * first matrix that brings the running total to k/g of the whole, or earlier
+ * when only one matrix remains for each later group; all-zero weights count
+ * matrices.  Returns g, or MUON_ERR_INVALID_ARG.  Host only.
+ */
+MUON_API int muon_offload_chunks(const long long* bytes, int count, int chunks, int* bounds);
+
 /* ---- per-shape coefficient schedules ----------------------------------------
  *
  * [ROOT] (staging.reportify.cn tag page, "ROOT优化器的技术创新"): the quintic

@@ -135,6 +135,46 @@ def muon_step(params, grads, momentum, mu=0.95, nesterov=True, lr=6e-4):
     _check(lib().muon_step(P, G, M, float(mu), 1 if nesterov else 0, float(lr), S, count))
 
 
+def _host_lane(host, dev, name):
+    """Pointers of the pinned host tensors that mirror the device tensors
+    `dev` (same shapes and dtypes), or None."""
+    if host is None:
+        return None
+    if len(host) != len(dev):
+        raise ValueError(f"{name} must have one tensor per parameter")
+    for h, d in zip(host, dev):
+        if h.is_cuda or not h.is_pinned():
+            raise ValueError(f"{name} must hold pinned (page-locked) host tensors")
+        if tuple(h.shape) != tuple(d.shape) or h.dtype != d.dtype or not h.is_contiguous():
+            raise ValueError(f"{name} tensors must be contiguous, with their device tensor's shape and dtype")
+    return (ctypes.c_void_p * len(host))(*[t.data_ptr() for t in host])
+
+
+def muon_step_offload(params, grads, momentum, grads_host=None, params_host=None, mu=0.95, nesterov=True,
+                      lr=6e-4, chunks=8):
+    """muon_step with the gradients copied in from pinned host tensors
+    (grads_host, into the device tensors grads) and the updated parameters
+    copied out to pinned host tensors (params_host), pipelined over `chunks`
+    groups of matrices so that the copies overlap the step."""
+    P, G, M, S, count = _muon_lane(params, grads, momentum)
+    GH = _host_lane(grads_host, grads, "grads_host")
+    PH = _host_lane(params_host, params, "params_host")
+    _bind_stream(params[0].device)
+    _check(lib().muon_step_offload(P, GH, G, M, PH, float(mu), 1 if nesterov else 0, float(lr), S, count,
+                                   int(chunks)))
+
+
+def muon_offload_chunks(weights, chunks):
+    """The grouping muon_step_offload uses: group bounds [0, ..., len(weights)]
+    of consecutive matrices with about equal total weight."""
+    count = len(weights)
+    W = (ctypes.c_longlong * max(count, 1))(*[int(w) for w in weights])
+    B = (ctypes.c_int * (max(min(chunks, count), 0) + 1))()
+    g = lib().muon_offload_chunks(W, count, int(chunks), B)
+    _check(min(g, 0))
+    return list(B[:g + 1])
+
+
 def muon_hybrid_step(params, grads, momentum, adam_params, adam_grads, exp_avg, exp_avg_sq, step,
                      mu=0.95, nesterov=True, lr=6e-4, adam_lr=6e-4, betas=(0.9, 0.95), eps=1e-8,
                      weight_decay=0.1):

@@ -41,7 +41,7 @@ EXPORTS = (
     "muon_profile_enable", "muon_profile_read", "muon_profile_reset",
     "muon_launch_count", "muon_normalize_noalloc", "muon_adamw_step",
     "muon_set_shape_coeffs", "muon_get_shape_coeffs", "muon_clear_shape_coeffs",
-    "muon_hybrid_step",
+    "muon_hybrid_step", "muon_step_offload", "muon_offload_chunks",
 )
 
 
@@ -129,6 +129,10 @@ def load(path=LIB_PATH):
         "muon_clear_shape_coeffs": (c_int, []),
         "muon_hybrid_step": (c_int, [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp), c_float, c_int,
                                      c_float, ctypes.POINTER(c_int), c_int, ctypes.POINTER(MuonAdamwLane)]),
+        "muon_step_offload": (c_int, [ctypes.POINTER(vp), ctypes.POINTER(vp), ctypes.POINTER(vp),
+                                      ctypes.POINTER(vp), ctypes.POINTER(vp), c_float, c_int, c_float,
+                                      ctypes.POINTER(c_int), c_int, c_int]),
+        "muon_offload_chunks": (c_int, [ctypes.POINTER(ctypes.c_longlong), c_int, c_int, ctypes.POINTER(c_int)]),
     }
     assert set(sig) == set(EXPORTS)
     for name, (res, args) in sig.items():

@@ -43,6 +43,13 @@ struct DeviceState {
     cudaEvent_t ws_event = nullptr;
     cudaStream_t ws_stream = nullptr;
     bool ws_used = false;
+    // muon_step_offload: one cached plan per group of matrices (the groups
+    // run back to back on the bound stream, so none rebuilds another's), and
+    // the two copy streams with their events (created on first use)
+    std::vector<std::unique_ptr<Plan>> chunk_plans;
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_out = nullptr;
+    std::vector<cudaEvent_t> ev_in, ev_done;  // per group: gradients landed, group stepped
 };
 std::deque<DeviceState> g_devs;  // deque: references stay valid on growth
 
@@ -233,11 +240,11 @@ struct AdamArgs {
     double bytes = 0;  // algorithmic HBM bytes
 };
 
-// Run the plan of rq (built or reused).  With `adam`, the AdamW lane's chunks
-// are appended to the grid of the plan's momentum launch.
-int run_plan(DeviceState* ds, const PlanRequest& rq, const AdamArgs* adam) {
+// Run rq with `plan` (built for it, or reused when its key matches).  With
+// `adam`, the AdamW lane's chunks are appended to the grid of the plan's
+// momentum launch.
+int run_plan(DeviceState* ds, Plan& plan, const PlanRequest& rq, const AdamArgs* adam) {
     std::string err;
-    Plan& plan = *ds->plan;
     int wst = ws_acquire(ds);
     if (wst != MUON_OK) return wst;
     if (!plan.same_shape_key(rq)) {
@@ -251,6 +258,7 @@ int run_plan(DeviceState* ds, const PlanRequest& rq, const AdamArgs* adam) {
         }
     }
     plan.set_scalars(rq.mu, rq.nesterov, rq.lr, rq.clip);
+    plan.set_index_base(rq.index_base);
     plan.set_adamw(adam ? &adam->L : nullptr, adam ? adam->bytes : 0.0);
     long long launched = 0;
     const int st = plan.run(g_stream, g_prof.on ? &g_prof : nullptr, &launched, err);
@@ -408,6 +416,66 @@ int check_device(DeviceState** ds, bool need_tc) {
     return MUON_OK;
 }
 
+// ---- muon_step_offload helpers ---------------------------------------------------
+
+// min(chunks, count) groups of consecutive matrices with about equal weight:
+// bounds[0] = 0 < bounds[1] < ... < bounds[g] = count.  Group k closes at the
+// first matrix that brings the running total to k/g of the whole, or earlier
+// when only one matrix remains for each group still to come.  Returns g.
+int offload_groups(const long long* bytes, int count, int chunks, int* bounds) {
+    const int g = std::min(chunks, count);
+    double total = 0;
+    for (int i = 0; i < count; ++i) total += static_cast<double>(bytes[i]);
+    const bool flat = !(total > 0);  // all zero: equal counts
+    if (flat) total = count;
+    bounds[0] = 0;
+    int k = 1;
+    double acc = 0;
+    for (int i = 0; i < count && k < g; ++i) {
+        acc += flat ? 1.0 : static_cast<double>(bytes[i]);
+        const int remain = count - (i + 1);
+        if (remain >= g - k && (acc * g >= total * k || remain == g - k)) bounds[k++] = i + 1;
+    }
+    bounds[k] = count;
+    return k;
+}
+
+// True for page-locked (pinned or registered) host memory.
+bool pinned_host(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeHost;
+}
+
+// The copy streams, events and plans of ds for `groups` groups (created once).
+int offload_resources(DeviceState* ds, int groups) {
+    cudaError_t e = cudaSuccess;
+    if (!ds->copy_in) e = cudaStreamCreateWithFlags(&ds->copy_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !ds->copy_out) e = cudaStreamCreateWithFlags(&ds->copy_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess && !ds->ev_start) e = cudaEventCreateWithFlags(&ds->ev_start, cudaEventDisableTiming);
+    if (e == cudaSuccess && !ds->ev_out) e = cudaEventCreateWithFlags(&ds->ev_out, cudaEventDisableTiming);
+    while (e == cudaSuccess && static_cast<int>(ds->ev_in.size()) < groups) {
+        cudaEvent_t a = nullptr, b = nullptr;
+        e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (a) cudaEventDestroy(a);
+            break;
+        }
+        ds->ev_in.push_back(a);
+        ds->ev_done.push_back(b);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(MUON_ERR_CUDA, std::string("copy stream or event creation failed: ") + cudaGetErrorString(e));
+    }
+    while (static_cast<int>(ds->chunk_plans.size()) < groups) ds->chunk_plans.emplace_back(new Plan());
+    return MUON_OK;
+}
+
 }  // namespace
 
 namespace muon {
@@ -459,6 +527,7 @@ int muon_release_workspace(void) {
             d.ws_used = false;
         }
         if (d.plan) d.plan->release();
+        for (auto& cp : d.chunk_plans) cp->release();
         if (d.adam_table) {
             cudaSetDevice(d.device);
             cudaFree(d.adam_table);
@@ -526,7 +595,7 @@ int muon_orthogonalize(int batch, int m, int n, void* X, const float* coeffs, in
     rq.restart_mask = g_cfg.restart_mask;
     rq.eps = g_cfg.eps;
     rq.device = ds->device;
-    return run_plan(ds, rq, nullptr);
+    return run_plan(ds, *ds->plan, rq, nullptr);
 }
 
 int muon_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov, float lr,
@@ -539,7 +608,7 @@ int muon_step(void* const* params, const void* const* grads, void* const* moment
     st = check_device(&ds, true);
     if (st != MUON_OK) return st;
     rq.device = ds->device;
-    return run_plan(ds, rq, nullptr);
+    return run_plan(ds, *ds->plan, rq, nullptr);
 }
 
 int muon_hybrid_step(void* const* params, const void* const* grads, void* const* momentum, float mu, int nesterov,
@@ -561,7 +630,96 @@ int muon_hybrid_step(void* const* params, const void* const* grads, void* const*
     if (st != MUON_OK) return st;
     st = adamw_upload(ds, aa);
     if (st != MUON_OK) return st;
-    return run_plan(ds, rq, &aa);
+    return run_plan(ds, *ds->plan, rq, &aa);
+}
+
+int muon_offload_chunks(const long long* bytes, int count, int chunks, int* bounds) {
+    if (count < 1 || chunks < 1) return fail(MUON_ERR_INVALID_ARG, "count and chunks must be >= 1");
+    if (!bytes || !bounds) return fail(MUON_ERR_INVALID_ARG, "bytes and bounds must not be NULL");
+    for (int i = 0; i < count; ++i)
+        if (bytes[i] < 0) return fail(MUON_ERR_INVALID_ARG, "bytes must be >= 0");
+    return offload_groups(bytes, count, chunks, bounds);
+}
+
+int muon_step_offload(void* const* params, const void* const* grads_host, void* const* grads, void* const* momentum,
+                      void* const* params_host, float mu, int nesterov, float lr, const int* shape_list, int count,
+                      int chunks) {
+    ensure_cfg();
+    if (chunks < 1) return fail(MUON_ERR_INVALID_ARG, "chunks must be >= 1");
+    PlanRequest whole;
+    int st = step_request(params, grads, momentum, mu, nesterov, lr, shape_list, count, whole);
+    if (st != MUON_OK) return st;
+    for (int i = 0; i < count; ++i)
+        if ((grads_host && !grads_host[i]) || (params_host && !params_host[i]))
+            return fail(MUON_ERR_INVALID_ARG, "null pointer in grads_host/params_host");
+    const size_t gsz = g_cfg.grad_dtype == MUON_DTYPE_F32 ? 4 : 2;
+    const size_t psz = g_cfg.param_dtype == MUON_DTYPE_F32 ? 4 : 2;
+    // groups of about equal copy bytes (both directions)
+    std::vector<long long> bytes(count);
+    for (int i = 0; i < count; ++i)
+        bytes[i] = static_cast<long long>(shape_list[2 * i]) * shape_list[2 * i + 1] *
+                   static_cast<long long>((grads_host ? gsz : 0) + (params_host ? psz : 0));
+    std::vector<int> bounds(std::min(chunks, count) + 1);
+    const int ngroups = offload_groups(bytes.data(), count, chunks, bounds.data());
+    std::vector<PlanRequest> rqs(ngroups);
+    for (int k = 0; k < ngroups; ++k) {
+        const int b = bounds[k], n = bounds[k + 1] - bounds[k];
+        st = step_request(params + b, grads + b, momentum + b, mu, nesterov, lr, shape_list + 2 * b, n, rqs[k]);
+        if (st != MUON_OK) return st;
+        rqs[k].index_base = b;
+    }
+    DeviceState* ds = nullptr;
+    st = check_device(&ds, true);
+    if (st != MUON_OK) return st;
+    for (int i = 0; i < count; ++i)
+        if ((grads_host && !pinned_host(grads_host[i])) || (params_host && !pinned_host(params_host[i])))
+            return fail(MUON_ERR_INVALID_ARG, "grads_host/params_host must be page-locked host memory");
+    st = offload_resources(ds, ngroups);
+    if (st != MUON_OK) return st;
+    auto elems = [&](int i) { return static_cast<size_t>(shape_list[2 * i]) * shape_list[2 * i + 1]; };
+    auto cuda_fail = [](cudaError_t e, const char* what) {
+        return fail(MUON_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+    };
+    // the copies start after the work already queued on the bound stream
+    cudaError_t e = cudaEventRecord(ds->ev_start, g_stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds->copy_in, ds->ev_start, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(ds->copy_out, ds->ev_start, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "stream ordering failed");
+    // every group's gradients, in order, on the host-to-device stream
+    if (grads_host) {
+        for (int k = 0; k < ngroups && e == cudaSuccess; ++k) {
+            for (int i = bounds[k]; i < bounds[k + 1] && e == cudaSuccess; ++i)
+                e = cudaMemcpyAsync(grads[i], grads_host[i], elems(i) * gsz, cudaMemcpyHostToDevice, ds->copy_in);
+            if (e == cudaSuccess) e = cudaEventRecord(ds->ev_in[k], ds->copy_in);
+        }
+    }
+    // the groups' steps on the bound stream, each followed by its copy out
+    int k = 0;
+    for (; k < ngroups && e == cudaSuccess; ++k) {
+        if (grads_host) {
+            e = cudaStreamWaitEvent(g_stream, ds->ev_in[k], 0);
+            if (e != cudaSuccess) break;
+        }
+        rqs[k].device = ds->device;
+        st = run_plan(ds, *ds->chunk_plans[k], rqs[k], nullptr);
+        if (st != MUON_OK) break;
+        if (params_host) {
+            e = cudaEventRecord(ds->ev_done[k], g_stream);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ds->copy_out, ds->ev_done[k], 0);
+            for (int i = bounds[k]; i < bounds[k + 1] && e == cudaSuccess; ++i)
+                e = cudaMemcpyAsync(params_host[i], params[i], elems(i) * psz, cudaMemcpyDeviceToHost, ds->copy_out);
+        }
+    }
+    const std::string run_err = st != MUON_OK ? g_err : std::string();
+    // join: work queued on the bound stream after this call follows every copy
+    cudaError_t j = cudaEventRecord(ds->ev_out, ds->copy_out);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(g_stream, ds->ev_out, 0);
+    if (j == cudaSuccess && grads_host) j = cudaEventRecord(ds->ev_out, ds->copy_in);
+    if (j == cudaSuccess && grads_host) j = cudaStreamWaitEvent(g_stream, ds->ev_out, 0);
+    if (st != MUON_OK) return fail(st, run_err);
+    if (e != cudaSuccess) return cuda_fail(e, "offload copy or ordering failed");
+    if (j != cudaSuccess) return cuda_fail(j, "stream join failed");
+    return MUON_OK;
 }
 
 int muon_set_shape_coeffs(int rows, int cols, const float* coeffs, int steps) {

@@ -396,6 +396,11 @@ void Plan::set_scalars(float mu, int nesterov, float lr, float clip) {
     }
 }
 
+void Plan::set_index_base(int base) {
+    for (LaunchRec& l : launches)
+        if (l.kind == LaunchRec::MOM) l.mom.mat_index_base = base;
+}
+
 void Plan::set_adamw(const AdamLaunch* adam, double bytes) {
     for (LaunchRec& l : launches)
         if (l.kind == LaunchRec::MOM) {

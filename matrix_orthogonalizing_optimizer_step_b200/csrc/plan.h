@@ -45,6 +45,7 @@ struct PlanRequest {
     float lr = 0.f;
     float clip = 0.f;              // muon_step: the update is clipped to [-clip, clip] (0 = off)
     int device = 0;
+    int index_base = 0;            // caller's index of matrix 0 (status reporting; per call, not in the key)
 };
 
 struct LaunchRec {
@@ -73,6 +74,9 @@ class Plan {
     bool same_shape_key(const PlanRequest& req) const;
     // Patch the per-call scalars (mu, nesterov, lr) into the launch records.
     void set_scalars(float mu, int nesterov, float lr, float clip);
+    // Patch the caller's index of matrix 0 (the first non-finite matrix is
+    // reported in the caller's numbering).
+    void set_index_base(int base);
     // Append (or, with null, remove) an AdamW lane to the momentum launch's
     // grid; `bytes` are its algorithmic HBM bytes (tracing).
     void set_adamw(const AdamLaunch* adam, double bytes);

@@ -172,3 +172,72 @@ def test_shape_schedule_table(lib):
     mo.muon_set_shape_coeffs(8, 8, [(2, 0, 0)])  # replacing an entry is still allowed when full
     mo.muon_reset_config()  # also clears the table
     assert mo.muon_get_shape_coeffs(8, 8) is None
+
+
+def test_offload_argument_errors(lib):
+    """muon_step_offload checks every argument before touching a device;
+    valid arguments on a host without a GPU give MUON_ERR_CUDA."""
+    vp = ctypes.c_void_p
+    P = (vp * 2)(0x1000, 0x2000)
+    Z = (vp * 2)(0x1000, None)
+    S = (ctypes.c_int * 4)(4, 4, 8, 8)
+    f = lib.muon_step_offload
+    assert f(P, P, P, P, P, 0.95, 1, 1e-3, S, 2, 0) == mo.MUON_ERR_INVALID_ARG     # chunks < 1
+    assert f(P, P, P, P, P, 0.95, 1, 1e-3, S, 0, 2) == mo.MUON_ERR_INVALID_ARG     # count < 1
+    assert f(P, Z, P, P, P, 0.95, 1, 1e-3, S, 2, 2) == mo.MUON_ERR_INVALID_ARG     # null host grad
+    assert f(P, P, P, P, Z, 0.95, 1, 1e-3, S, 2, 2) == mo.MUON_ERR_INVALID_ARG     # null host param
+    assert f(P, P, Z, P, P, 0.95, 1, 1e-3, S, 2, 2) == mo.MUON_ERR_INVALID_ARG     # null device grad
+    assert f(P, P, P, P, P, float("nan"), 1, 1e-3, S, 2, 2) == mo.MUON_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():
+        assert f(P, P, P, P, P, 0.95, 1, 1e-3, S, 2, 2) == mo.MUON_ERR_CUDA
+        assert f(P, None, P, P, None, 0.95, 1, 1e-3, S, 2, 1) == mo.MUON_ERR_CUDA
+
+
+def _groups_by_definition(w, chunks):
+    """The grouping rule stated in include/muon.h, applied by search: each
+    bound is the first index after the previous one at which the running
+    total reaches k/g of the whole (while a matrix remains for every later
+    group), or at which only one matrix remains per later group."""
+    n, g = len(w), min(chunks, len(w))
+    if sum(w) == 0:
+        w = [1] * n
+    total = sum(w)
+    bounds = [0]
+    for k in range(1, g):
+        cands = [j for j in range(bounds[-1] + 1, n + 1)
+                 if n - j >= g - k and (sum(w[:j]) * g >= total * k or n - j == g - k)]
+        bounds.append(cands[0])
+    return bounds + [n]
+
+
+def test_offload_grouping(lib):
+    import random
+    rng = random.Random(7)
+    assert mo.muon_offload_chunks([10] * 8, 4) == [0, 2, 4, 6, 8]
+    assert mo.muon_offload_chunks([1, 1, 1, 100], 4) == [0, 1, 2, 3, 4]   # a heavy tail still splits
+    assert mo.muon_offload_chunks([5], 8) == [0, 1]
+    assert mo.muon_offload_chunks([0, 0, 0], 2) == [0, 2, 3]             # all-zero weights count matrices
+    for _ in range(300):
+        n = rng.randint(1, 40)
+        w = [rng.choice([0, 1, 7, 1000, rng.randint(0, 10 ** 9)]) for _ in range(n)]
+        c = rng.randint(1, 12)
+        b = mo.muon_offload_chunks(w, c)
+        assert len(b) == min(c, n) + 1 and b[0] == 0 and b[-1] == n
+        assert all(x < y for x, y in zip(b, b[1:]))
+        assert b == _groups_by_definition(w, c), (w, c)
+    # equal weights split evenly; a real layer set splits at layer bounds
+    layer = [4096 * 4096, 1024 * 4096, 1024 * 4096, 4096 * 4096, 14336 * 4096, 14336 * 4096, 4096 * 14336]
+    assert mo.muon_offload_chunks(layer * 32, 8) == list(range(0, 225, 28))
+    for bad in [([1], 0), ([], 2), ([-1, 2], 2)]:
+        with pytest.raises(mo.MuonError):
+            mo.muon_offload_chunks(*bad)
+
+
+def test_offload_binding_validates_host_tensors():
+    import torch
+    a = torch.zeros(4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mo.muon_step_offload([a], [a], [a], grads_host=[a, a])   # one host tensor per parameter
+    with pytest.raises(ValueError):
+        mo.muon_step_offload([a], [a], [a], params_host=[a])     # not pinned

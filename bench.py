@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--form", default="auto", choices=["auto", "standard", "gram"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--offload-chunks", type=int, default=8,
+    ap.add_argument("--offload-chunks", type=int, default=16,
                     help="groups of matrices the e2e leg's offload step pipelines its copies over")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-adamw", action="store_true",

@@ -489,7 +489,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
         // Local copies: the epilogue stores to global memory, so fields read
         // through a reference into the problem table would be reloaded after
         // every store (the compiler cannot rule out aliasing).
-        const Epilogue ep = L.problems[tile.problem].ep;
+        Epilogue ep = L.problems[tile.problem].ep;
         const int PM = L.problems[tile.problem].M, PN = L.problems[tile.problem].N;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
         // the epilogue inputs (C1) come from earlier slots: acquire them too
@@ -524,6 +524,13 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             const int bytes = min(S::cols, PN - cbase) * es;
             for (int o = 0; o < bytes; o += 128) prefetch_l2(p + o);
         }
+        // The fused update of fp32 parameters, W <- W + d in place (C2 = the
+        // output, coefficient 1): the warp stages d alone and the TMA store
+        // adds it to W at L2, so W is never loaded into registers.  The sum
+        // is the one rounding of W + d that the register path makes.
+        const bool radd = use_tma && ep.c2 != nullptr && ep.c2 == ep.o1 && ep.ldc2 == ep.ldo1 &&
+                          ep.c2_dt == DT_F32 && ep.o1_dt == DT_F32 && ep.gamma == 1.f;
+        if (radd) ep.c2 = nullptr;
         // every lane waits; the warp leaves together unless all lanes saw the
         // accumulator arrive (a lane's wait may end just before the arrival)
         const bool got = mbar_wait(&sh->tfull[acc], acc_phase, abort_flag, lim);
@@ -588,7 +595,10 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
                 fence_proxy_async_shared();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(omap, buf, col0 + 16 * h, static_cast<int>(row0), ep.o1_z);
+                    if (radd)
+                        tma_reduce_add_3d(omap, buf, col0 + 16 * h, static_cast<int>(row0), ep.o1_z);
+                    else
+                        tma_store_3d(omap, buf, col0 + 16 * h, static_cast<int>(row0), ep.o1_z);
                     bulk_commit();
                 }
                 ++nstored;

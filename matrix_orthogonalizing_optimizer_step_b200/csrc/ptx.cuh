@@ -207,6 +207,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t sm
                  : "memory");
 }
 
+// Add a staged box element-wise into the tensor in global memory (the add
+// runs at L2; the element type is the tensor map's).  Out-of-range rows and
+// columns are clipped as for a store.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t smem_src, int c0, int c1, int c2) {
+    asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];"
+                 ::"l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_src)
+                 : "memory");
+}
+
 // Pull the 128-byte line holding `p` into L2 (no register result).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));

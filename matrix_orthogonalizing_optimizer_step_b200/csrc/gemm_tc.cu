@@ -525,11 +525,15 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             for (int o = 0; o < bytes; o += 128) prefetch_l2(p + o);
         }
         // The fused update of fp32 parameters, W <- W + d in place (C2 = the
-        // output, coefficient 1): the warp stages d alone and the TMA store
-        // adds it to W at L2, so W is never loaded into registers.  The sum
-        // is the one rounding of W + d that the register path makes.
-        const bool radd = use_tma && ep.c2 != nullptr && ep.c2 == ep.o1 && ep.ldc2 == ep.ldo1 &&
-                          ep.c2_dt == DT_F32 && ep.o1_dt == DT_F32 && ep.gamma == 1.f;
+        // output, coefficient 1), in chained launches: the warp stages d alone
+        // and the TMA store adds it to W at L2, so W is never loaded into
+        // registers and the accumulator is released sooner (the epilogue is
+        // the limit there).  The sum is the one rounding of W + d that the
+        // register path makes.  Persistent launches keep the register path:
+        // their limit is the operand feed from L2, which the adds at L2 would
+        // compete with.
+        const bool radd = GROUPS == kChainGroups && use_tma && ep.c2 != nullptr && ep.c2 == ep.o1 &&
+                          ep.ldc2 == ep.ldo1 && ep.c2_dt == DT_F32 && ep.o1_dt == DT_F32 && ep.gamma == 1.f;
         if (radd) ep.c2 = nullptr;
         // every lane waits; the warp leaves together unless all lanes saw the
         // accumulator arrive (a lane's wait may end just before the arrival)

@@ -33,6 +33,14 @@
  *    streams: a call's use of the workspace is ordered after the previous
  *    call's, on whichever stream that ran (an event wait, not a host sync).
  *    The caller's own tensors are not synchronised across streams.
+ *  - CUDA graphs: muon_step, muon_orthogonalize, muon_adamw_step and
+ *    muon_hybrid_step may be captured (stream capture of the bound stream)
+ *    once the same call has run before the capture: a capture never builds
+ *    a plan or uploads a table (MUON_ERR_UNSUPPORTED, nothing enqueued, if it
+ *    would have to).  Under capture the cross-stream workspace ordering is
+ *    left to the capture and the graph's launches.  Scalars (mu, lr, the
+ *    AdamW step count and its bias corrections) are launch arguments: a
+ *    graph replays the values it was captured with.
  *  - Every call returns a status (< 0 on error) and never throws.  On an
  *    argument error nothing is enqueued; muon_last_error() describes it.
  *  - Every device-side wait (a CTA pair waiting for its operands, for another

@@ -215,8 +215,22 @@ struct Profiler : ProfileSink {
 };
 Profiler g_prof;
 
+// True while the bound stream is being captured into a CUDA graph.
+bool capturing() {
+    cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(g_stream, &st) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return st != cudaStreamCaptureStatusNone;
+}
+
 // Order this call's use of the workspace after its last use on another stream.
+// Under stream capture the ordering belongs to the capture (it starts after
+// the work it was forked from) and to the graph's launches, so no event of
+// an earlier, uncaptured call is waited on.
 int ws_acquire(DeviceState* ds) {
+    if (capturing()) return MUON_OK;
     if (ds->ws_used && ds->ws_stream != g_stream) {
         const cudaError_t e = cudaStreamWaitEvent(g_stream, ds->ws_event, 0);
         if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("stream wait failed: ") + cudaGetErrorString(e));
@@ -224,8 +238,10 @@ int ws_acquire(DeviceState* ds) {
     return MUON_OK;
 }
 
-// Mark the end of this call's use of the workspace on the bound stream.
+// Mark the end of this call's use of the workspace on the bound stream (not
+// under stream capture: the captured launches run when the graph does).
 int ws_release(DeviceState* ds) {
+    if (capturing()) return MUON_OK;
     const cudaError_t e = cudaEventRecord(ds->ws_event, g_stream);
     if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("event record failed: ") + cudaGetErrorString(e));
     ds->ws_stream = g_stream;
@@ -245,6 +261,12 @@ struct AdamArgs {
 // momentum launch.
 int run_plan(DeviceState* ds, Plan& plan, const PlanRequest& rq, const AdamArgs* adam) {
     std::string err;
+    // a plan is built with allocations, uploads and a stream synchronisation,
+    // none of which a stream capture allows: capture only calls whose plan
+    // exists (the same call made once before the capture)
+    if (capturing() && !plan.same_shape_key(rq))
+        return fail(MUON_ERR_UNSUPPORTED,
+                    "stream capture needs a built plan: make the same call once before capturing it");
     int wst = ws_acquire(ds);
     if (wst != MUON_OK) return wst;
     if (!plan.same_shape_key(rq)) {
@@ -382,6 +404,10 @@ int adamw_upload(DeviceState* ds, AdamArgs& aa) {
     std::vector<AdamTensor>& last = ds->adam_last;
     const std::vector<AdamTensor>& t = aa.t;
     const size_t bytes = sizeof(AdamTensor) * t.size();
+    const bool same = last.size() == t.size() && std::memcmp(last.data(), t.data(), bytes) == 0;
+    if (!same && capturing())
+        return fail(MUON_ERR_UNSUPPORTED,
+                    "stream capture needs the AdamW table in place: make the same call once before capturing it");
     if (ds->adam_cap < bytes) {
         if (ds->adam_table) {
             cudaStreamSynchronize(g_stream);
@@ -399,7 +425,7 @@ int adamw_upload(DeviceState* ds, AdamArgs& aa) {
         ds->adam_cap = bytes;
         last.clear();
     }
-    if (last.size() != t.size() || std::memcmp(last.data(), t.data(), bytes) != 0) {
+    if (!same) {
         cudaError_t e = cudaMemcpyAsync(ds->adam_table, t.data(), bytes, cudaMemcpyHostToDevice, g_stream);
         if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table upload failed: ") + cudaGetErrorString(e));
         last = t;

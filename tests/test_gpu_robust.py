@@ -183,3 +183,57 @@ def test_calls_alternating_streams():
     st, _ = mo.muon_device_status()
     assert st == mo.MUON_OK
     assert np.all(np.isfinite(to64(got[0])))
+
+
+@pytest.mark.parametrize("env", [{}, {"MUON_SLOT_LAUNCHES": "1"}])
+def test_step_captured_in_a_cuda_graph(env, monkeypatch):
+    """A muon_step captured into a CUDA graph (after one eager call built its
+    plan) and replayed three times equals four eager steps bit for bit, in
+    the chained launch and with one launch per chain slot."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    mo.muon_release_workspace()  # the launch mode is chosen when a plan is built
+    shapes = [(768, 2304), (768, 768), (3072, 768), (200, 712)]
+    G = [wl.make_single(r, c, 700 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, 710 + i, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, 720 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    Wr, Mr = [t.clone() for t in W], [t.clone() for t in M]
+    for _ in range(4):
+        mo.muon_step(Wr, G, Mr, lr=0.02)
+    torch.cuda.synchronize()
+    mo.muon_step(W, G, M, lr=0.02)  # builds the plan of (W, G, M)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        mo.muon_step(W, G, M, lr=0.02)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(W + M, Wr + Mr):
+        assert torch.equal(a, b)
+    del graph
+    mo.muon_release_workspace()
+
+
+@pytest.mark.filterwarnings("ignore:The CUDA Graph is empty")  # the refused capture enqueued nothing
+def test_capture_that_needs_a_plan_is_refused():
+    """Capturing a call whose plan does not exist yet fails with
+    MUON_ERR_UNSUPPORTED before anything is enqueued (building a plan
+    allocates and synchronises, which a capture does not allow)."""
+    mo.muon_release_workspace()
+    W = [wl.make_single(256, 512, 730, "params", DEV, "f32")]
+    G = [wl.make_single(256, 512, 731, "student_t3", DEV, "bf16", 0.01)]
+    M = [wl.make_single(256, 512, 732, "student_t3", DEV, "bf16", 0.01)]
+    W0 = W[0].clone()
+    graph = torch.cuda.CUDAGraph()
+    with pytest.raises(mo.MuonError) as e:
+        with torch.cuda.graph(graph):
+            mo.muon_step(W, G, M, lr=0.02)
+    assert e.value.code == mo.MUON_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.equal(W[0], W0)
+    del graph
+    # outside a capture the same call builds its plan and runs
+    mo.muon_step(W, G, M, lr=0.02)
+    torch.cuda.synchronize()
+    assert not torch.equal(W[0], W0)

@@ -62,6 +62,8 @@ def parse():
                     help="with N > 1: one independent replica of the workload per GPU instead of the sharded step")
     ap.add_argument("--also", default="2",
                     help="comma-separated workload ids timed on the device after the main one (extra key)")
+    ap.add_argument("--no-spectral", action="store_true",
+                    help="skip the singular-value report of orthogonalised updates")
     ap.add_argument("--subset", type=int, default=0,
                     help="use only the first N matrices of the workload (small profiling cases)")
     return ap.parse_args()
@@ -422,6 +424,36 @@ def gemm_roofline(prof, ms_total, ms_per_step, peaks, peak_src, traffic):
     }
 
 
+def spectral_report(w, dev, form):
+    """Singular values after the Newton-Schulz iteration, the monitoring check
+    of [NanoGPT-Muon] "落地监控指标" (they should sit near 1): the gradient of
+    the first matrix of each distinct shape, orthogonalised by the library
+    (muon_orthogonalize, 5 tuned steps, the step's form), then torch's svdvals
+    in fp32.  Outside every timed region.  The tuned coefficients map input
+    singular values of at least 3e-3 (normalised) into [0.68, 1.21]; smaller
+    ones stay below (the iteration's small-sigma gain is a^5 ~ 487)."""
+    import torch
+    import matrix_orthogonalizing_optimizer_step_b200 as mo
+    out = []
+    seen = set()
+    for i, shape in enumerate(w.shapes):
+        if shape in seen:
+            continue
+        seen.add(shape)
+        x = wl.make_matrix(w, i, wl.ROLE_GRAD, device=dev, dtype="bf16").contiguous()
+        mo.muon_orthogonalize(x, steps=5, mode=form)
+        sv = torch.linalg.svdvals(x.float())
+        q = torch.quantile(sv, torch.tensor([0.01, 0.5, 0.99], device=sv.device)).tolist()
+        out.append({"shape": list(shape), "sigma_min": round(float(sv.min()), 4),
+                    "sigma_p01": round(q[0], 4), "sigma_p50": round(q[1], 4), "sigma_p99": round(q[2], 4),
+                    "sigma_max": round(float(sv.max()), 4),
+                    "frac_in_0.68_1.21": round(float(((sv >= 0.68) & (sv <= 1.21)).float().mean()), 4)})
+        del x, sv
+    torch.cuda.empty_cache()
+    mo.muon_release_workspace()
+    return {"check": "singular values of orthogonalised gradients (first matrix of each shape)", "shapes": out}
+
+
 def measure_extra(w, dev, args, peaks, peak_src, world):
     """Device-timed step of another workload (no e2e, no CPU leg)."""
     import torch
@@ -637,6 +669,10 @@ def run_ours(args):
         ew = wl.WORKLOADS[wid]
         extra[ew.name] = measure_extra(ew, dev, args, peaks, peak_src, world)
 
+    spectral = None
+    if world == 1 and not args.no_spectral:
+        spectral = spectral_report(w, dev, args.form)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample = cpu_oracle_step_ms(w, args.cpu_seconds, args.form, args.soft_threshold)
@@ -665,6 +701,7 @@ def run_ours(args):
             "e2e": e2e, "cpu_baseline": cpu, "clocks": clk,
             "adamw_lane": adamw,
             "hybrid_lane": hybrid,
+            "spectral": spectral,
             "also": extra,
         }
         print(json.dumps(out), flush=True)

@@ -58,6 +58,11 @@
  *    MUON_CHAIN_LAUNCH / MUON_SLOT_LAUNCHES  force one launch for the whole
  *                        Newton-Schulz chain / one launch per chain slot
  *    MUON_TMA_STORE=0    plain per-lane stores in the GEMM epilogue
+ *    MUON_DEBUG_CANARY=1 every workspace region is followed by a 1 KB guard
+ *                        of a fixed byte pattern; after each call's launches
+ *                        a check kernel compares every guard with it (and
+ *                        restores it), so muon_device_status returns
+ *                        MUON_ERR_GUARD after a write past a region's end
  *    MUON_PROFILE_VERBOSE  print every traced launch to stderr
  */
 #ifndef MUON_B200_H
@@ -83,6 +88,7 @@ extern "C" {
 #define MUON_ERR_NO_MEMORY (-4)   /* workspace allocation failed */
 #define MUON_ERR_TIMEOUT (-5)     /* a bounded device-side wait ran out */
 #define MUON_ERR_NONFINITE (-6)   /* ||U||_F was not finite for some matrix */
+#define MUON_ERR_GUARD     (-7)   /* debug canary mode: a workspace guard was overwritten */
 
 /* mode bits of muon_orthogonalize and muon_config.mode */
 #define MUON_NS_STANDARD 0  /* A = X X^T, B = bA + cA^2, X <- aX + BX          */
@@ -274,6 +280,15 @@ MUON_API int muon_hybrid_step(void* const* params, const void* const* grads, voi
 MUON_API int muon_step_offload(void* const* params, const void* const* grads_host, void* const* grads,
                                void* const* momentum, void* const* params_host, float mu, int nesterov, float lr,
                                const int* shape_list, int count, int chunks);
+
+/*
+ * muon_debug_corrupt_guard -- debug canary mode only: overwrite one byte of
+ * workspace guard `index` of the current plan (a plain memset on the bound
+ * stream, inside the library's own allocation), so that a test can see the
+ * next call's check report MUON_ERR_GUARD.  MUON_ERR_INVALID_ARG when the
+ * mode is off, no plan exists or the index is out of range.
+ */
+MUON_API int muon_debug_corrupt_guard(int index);
 
 /*
  * muon_offload_chunks -- the grouping of muon_step_offload: with bytes[i] >= 0

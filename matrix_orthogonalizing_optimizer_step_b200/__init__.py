@@ -12,7 +12,7 @@ import ctypes
 
 from . import _lib
 from ._lib import (  # noqa: F401
-    MUON_DTYPE_BF16, MUON_DTYPE_F32, MUON_ERR_CUDA, MUON_ERR_INVALID_ARG,
+    MUON_DTYPE_BF16, MUON_DTYPE_F32, MUON_ERR_CUDA, MUON_ERR_GUARD, MUON_ERR_INVALID_ARG,
     MUON_ERR_NO_MEMORY, MUON_ERR_NONFINITE, MUON_ERR_TIMEOUT,
     MUON_ERR_UNSUPPORTED, MUON_MAX_SHAPE_SCHEDULES, MUON_MAX_STEPS, MUON_NS_AUTO, MUON_NS_GRAM,
     MUON_NS_STANDARD, MUON_OK, MUON_PREC_FP32, STATUS_NAMES,
@@ -293,6 +293,14 @@ def muon_device_status(device=None):
     bad = ctypes.c_int(-1)
     rc = lib().muon_device_status(ctypes.byref(bad))
     return rc, bad.value
+
+
+def muon_debug_corrupt_guard(index, device=None):
+    """Debug canary mode (MUON_DEBUG_CANARY=1): overwrite one byte of a
+    workspace guard of the current plan, for tests of the guard check."""
+    import torch
+    _bind_stream(device if device is not None else torch.cuda.current_device())
+    _check(lib().muon_debug_corrupt_guard(int(index)))
 
 
 def muon_release_workspace():

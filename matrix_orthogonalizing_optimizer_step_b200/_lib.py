@@ -14,6 +14,7 @@ MUON_ERR_CUDA = -3
 MUON_ERR_NO_MEMORY = -4
 MUON_ERR_TIMEOUT = -5
 MUON_ERR_NONFINITE = -6
+MUON_ERR_GUARD = -7
 
 MUON_NS_STANDARD = 0
 MUON_NS_GRAM = 1
@@ -30,7 +31,7 @@ STATUS_NAMES = {
     MUON_OK: "MUON_OK", MUON_ERR_INVALID_ARG: "MUON_ERR_INVALID_ARG",
     MUON_ERR_UNSUPPORTED: "MUON_ERR_UNSUPPORTED", MUON_ERR_CUDA: "MUON_ERR_CUDA",
     MUON_ERR_NO_MEMORY: "MUON_ERR_NO_MEMORY", MUON_ERR_TIMEOUT: "MUON_ERR_TIMEOUT",
-    MUON_ERR_NONFINITE: "MUON_ERR_NONFINITE",
+    MUON_ERR_NONFINITE: "MUON_ERR_NONFINITE", MUON_ERR_GUARD: "MUON_ERR_GUARD",
 }
 
 # every symbol include/muon.h declares
@@ -41,7 +42,7 @@ EXPORTS = (
     "muon_profile_enable", "muon_profile_read", "muon_profile_reset",
     "muon_launch_count", "muon_normalize_noalloc", "muon_adamw_step",
     "muon_set_shape_coeffs", "muon_get_shape_coeffs", "muon_clear_shape_coeffs",
-    "muon_hybrid_step", "muon_step_offload", "muon_offload_chunks",
+    "muon_hybrid_step", "muon_step_offload", "muon_offload_chunks", "muon_debug_corrupt_guard",
 )
 
 
@@ -133,6 +134,7 @@ def load(path=LIB_PATH):
                                       ctypes.POINTER(vp), ctypes.POINTER(vp), c_float, c_int, c_float,
                                       ctypes.POINTER(c_int), c_int, c_int]),
         "muon_offload_chunks": (c_int, [ctypes.POINTER(ctypes.c_longlong), c_int, c_int, ctypes.POINTER(c_int)]),
+        "muon_debug_corrupt_guard": (c_int, [c_int]),
     }
     assert set(sig) == set(EXPORTS)
     for name, (res, args) in sig.items():

@@ -107,6 +107,10 @@ struct MomLaunch {
 };
 cudaError_t launch_momentum_norm(const MomLaunch& L, cudaStream_t stream);
 
+// Debug canary mode: check (and re-arm) the n workspace guards at base + offs[i].
+cudaError_t launch_guard_check(void* base, const unsigned long long* offs, int n, DeviceStatus* status,
+                               cudaStream_t stream);
+
 struct ScaleLaunch {
     const ScaleMatrix* mats;
     int nmats;

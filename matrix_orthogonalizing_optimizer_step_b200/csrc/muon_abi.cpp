@@ -2,6 +2,7 @@
 // stream binding, the device status word, tracing, and the two entry points.
 // No exception crosses this boundary; every entry point returns a status.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -579,6 +580,8 @@ int muon_device_status(int* bad_index) {
     const DeviceStatus init{0, 0x7fffffff};
     cudaMemcpy(ds->status, &init, sizeof(init), cudaMemcpyHostToDevice);
     if (bad_index && h.first_bad != 0x7fffffff) *bad_index = h.first_bad;
+    if (h.bits & ST_GUARD)
+        return fail(MUON_ERR_GUARD, "a workspace guard was overwritten (a write past the end of a workspace region)");
     if (h.bits & ST_TIMEOUT) return fail(MUON_ERR_TIMEOUT, "a kernel's bounded wait ran out");
     if (h.bits & ST_NONFINITE) return fail(MUON_ERR_NONFINITE, "non-finite Frobenius norm");
     return MUON_OK;
@@ -659,6 +662,19 @@ int muon_hybrid_step(void* const* params, const void* const* grads, void* const*
     return run_plan(ds, *ds->plan, rq, &aa);
 }
 
+int muon_debug_corrupt_guard(int index) {
+    if (index < 0) return fail(MUON_ERR_INVALID_ARG, "index must be >= 0");
+    DeviceState* ds = nullptr;
+    const int st = device_state(&ds);
+    if (st != MUON_OK) return st;
+    if (index >= ds->plan->guard_count())
+        return fail(MUON_ERR_INVALID_ARG, "no such guard (MUON_DEBUG_CANARY=1 and a plan built by muon_step or "
+                                          "muon_orthogonalize are needed)");
+    const cudaError_t e = cudaMemsetAsync(ds->plan->guard_addr(index), 0, 1, g_stream);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("memset failed: ") + cudaGetErrorString(e));
+    return MUON_OK;
+}
+
 int muon_offload_chunks(const long long* bytes, int count, int chunks, int* bounds) {
     if (count < 1 || chunks < 1) return fail(MUON_ERR_INVALID_ARG, "count and chunks must be >= 1");
     if (!bytes || !bounds) return fail(MUON_ERR_INVALID_ARG, "bytes and bounds must not be NULL");
@@ -727,7 +743,11 @@ int muon_step_offload(void* const* params, const void* const* grads_host, void* 
             if (e != cudaSuccess) break;
         }
         rqs[k].device = ds->device;
+        char label[40];
+        std::snprintf(label, sizeof(label), "muon offload group %d", k);
+        nvtxRangePushA(label);
         st = run_plan(ds, *ds->chunk_plans[k], rqs[k], nullptr);
+        nvtxRangePop();
         if (st != MUON_OK) break;
         if (params_host) {
             e = cudaEventRecord(ds->ev_done[k], g_stream);
@@ -806,7 +826,9 @@ int muon_adamw_step(void* const* params, const void* const* grads, void* const* 
     st = adamw_upload(ds, aa);
     if (st != MUON_OK) return st;
     if (g_prof.on) g_prof.before(g_stream);
+    nvtxRangePushA("muon adamw");
     cudaError_t e = launch_adamw(aa.L, g_stream);
+    nvtxRangePop();
     if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("kernel launch failed: ") + cudaGetErrorString(e));
     ++g_launches;
     if (g_prof.on) g_prof.after(g_stream, 4, 0.0, aa.bytes);

@@ -10,7 +10,11 @@ enum DType : int { DT_BF16 = 0, DT_F32 = 1, DT_F16 = 2 };
 inline int dtype_size(int dt) { return dt == DT_F32 ? 4 : 2; }
 
 // device status word bits
-enum : int { ST_TIMEOUT = 1, ST_NONFINITE = 2 };
+enum : int { ST_TIMEOUT = 1, ST_NONFINITE = 2, ST_GUARD = 4 };
+
+// Workspace guards of the debug canary mode (MUON_DEBUG_CANARY=1).
+constexpr int kGuardBytes = 1024;
+constexpr unsigned char kGuardByte = 0xA5;
 
 struct DeviceStatus {
     int bits;       // ST_* flags, sticky until read by the host

@@ -19,7 +19,10 @@
 // product accumulates in fp32 and every stored matrix is rounded once.
 #include "plan.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 #include <algorithm>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <map>
@@ -80,6 +83,11 @@ int fault_mode() {
     if (!std::strcmp(f, "launch")) return FAULT_LAUNCH;
     if (!std::strcmp(f, "timeout")) return FAULT_TIMEOUT;
     return FAULT_NONE;
+}
+
+bool canary_mode() {
+    const char* v = std::getenv("MUON_DEBUG_CANARY");
+    return v && v[0] == '1';
 }
 
 // Bound of every device-side wait (MUON_WAIT_LIMIT_MS, 1 ms .. 10 s; default 1 s).
@@ -370,6 +378,7 @@ static std::vector<long long> make_key(const PlanRequest& rq) {
     }
     for (int si : rq.sched) k.push_back(si);
     k.push_back(fault_mode());
+    k.push_back(canary_mode() ? 1 : 0);
     k.push_back(static_cast<long long>(wait_limit_ns()));
     for (size_t i = 0; i < rq.rows.size(); ++i) {
         k.push_back(rq.rows[i]);
@@ -419,6 +428,8 @@ void Plan::release() {
     arena_bytes = 0;
     launches.clear();
     key_.clear();
+    guard_offs_.clear();
+    d_guard_offs_ = nullptr;
 }
 
 int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaStream_t stream, std::string& err) {
@@ -492,10 +503,19 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     }
 
     // ---- workspace layout --------------------------------------------------------
+    // Regions start 1024-byte aligned.  In the debug canary mode each region
+    // is followed, from its exact end, by a guard of kGuardBytes.
+    const bool canary = canary_mode();
+    guard_offs_.clear();
     size_t cursor = 0;
     auto take = [&](size_t bytes) {
         const size_t o = cursor;
-        cursor = static_cast<size_t>(round_up(static_cast<long long>(cursor + bytes), 1024));
+        size_t end = o + bytes;
+        if (canary) {
+            guard_offs_.push_back(end);
+            end += kGuardBytes;
+        }
+        cursor = static_cast<size_t>(round_up(static_cast<long long>(end), 1024));
         return o;
     };
     for (Group& g : groups) {
@@ -561,6 +581,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     // TMA store maps: one per workspace buffer of a group, one per caller output
     nmaps_max += groups.size() * NBUF + static_cast<size_t>(nm);
     const size_t off_maps = take(sizeof(CUtensorMap) * std::max<size_t>(nmaps_max, 1));
+    // the guard offsets, themselves guarded (their own entry is the last one)
+    const size_t off_guards = canary ? take(sizeof(unsigned long long) * (guard_offs_.size() + 1)) : 0;
     const size_t need = cursor;
 
     // ---- arena -----------------------------------------------------------------
@@ -581,6 +603,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         arena_bytes = need;
     }
     char* base = static_cast<char*>(arena_);
+    status_ = status;
+    d_guard_offs_ = canary ? reinterpret_cast<const unsigned long long*>(base + off_guards) : nullptr;
     float* d_partials = reinterpret_cast<float*>(base + off_partials);
     int* d_counters = reinterpret_cast<int*>(base + off_counters);
     float* d_scale = reinterpret_cast<float*>(base + off_scale);
@@ -637,6 +661,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     {
         LaunchRec lr;
         lr.kind = LaunchRec::MOM;
+        std::snprintf(lr.label, sizeof(lr.label), "muon momentum+norm");
         MomLaunch& L = lr.mom;
         L.mats = reinterpret_cast<const MomMatrix*>(base + off_moms);
         L.nmats = nm;
@@ -689,6 +714,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         }
         LaunchRec lr;
         lr.kind = LaunchRec::SCALE;
+        std::snprintf(lr.label, sizeof(lr.label), "muon scale");
         ScaleLaunch& L = lr.sc;
         L.mats = reinterpret_cast<const ScaleMatrix*>(base + off_smats);
         L.nmats = static_cast<int>(smats.size());
@@ -722,6 +748,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     }
     LaunchRec chain;
     chain.kind = LaunchRec::TC;
+    std::snprintf(chain.label, sizeof(chain.label), "muon gemm chain");
     bool chain_open = false;
     std::vector<CUtensorMap> maps;
     std::map<std::tuple<int, int, int>, int> map_index;  // (group, buf, box kind)
@@ -813,6 +840,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     for (size_t si = 0; si < nslots; ++si) {
         LaunchRec lr;
         lr.kind = f32 ? LaunchRec::F32 : LaunchRec::TC;
+        std::snprintf(lr.label, sizeof(lr.label), f32 ? "muon gemm_f32 slot %zu" : "muon gemm slot %zu", si);
         const size_t prob_begin = f32 ? fprobs.size() : tprobs.size();
         const size_t tile_begin = tiles.size();
         struct TileRef {
@@ -1038,6 +1066,12 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     if (e == cudaSuccess && !maps.empty()) e = up(off_maps, maps.data(), sizeof(CUtensorMap) * maps.size());
     if (e == cudaSuccess) e = cudaMemsetAsync(d_counters, 0, sizeof(int) * nm, stream);
     if (e == cudaSuccess) e = cudaMemsetAsync(d_done, 0, sizeof(unsigned) * nm, stream);
+    if (canary) {
+        if (e == cudaSuccess)
+            e = up(off_guards, guard_offs_.data(), sizeof(unsigned long long) * guard_offs_.size());
+        for (size_t i = 0; i < guard_offs_.size() && e == cudaSuccess; ++i)
+            e = cudaMemsetAsync(base + guard_offs_[i], kGuardByte, kGuardBytes, stream);
+    }
     if (e != cudaSuccess) {
         err = std::string("table upload failed: ") + cudaGetErrorString(e);
         return MUON_ERR_CUDA;
@@ -1052,6 +1086,8 @@ int Plan::run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter,
         return MUON_ERR_CUDA;
     }
     for (const LaunchRec& lr : launches) {
+        // one NVTX range per launch (host-side enqueue, named by phase and slot)
+        nvtxRangePushA(lr.label);
         if (prof) prof->before(stream);
         cudaError_t e = cudaSuccess;
         switch (lr.kind) {
@@ -1060,12 +1096,21 @@ int Plan::run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter,
             case LaunchRec::TC: e = launch_gemm_tc(lr.tc, lr.grid, stream); break;
             case LaunchRec::F32: e = launch_gemm_f32(lr.f32, stream); break;
         }
+        nvtxRangePop();
         if (e != cudaSuccess) {
             err = std::string("kernel launch failed: ") + cudaGetErrorString(e);
             return MUON_ERR_CUDA;
         }
         if (launch_counter) ++*launch_counter;
         if (prof) prof->after(stream, static_cast<int>(lr.kind), lr.flops, lr.bytes + lr.extra_bytes);
+    }
+    if (d_guard_offs_) {  // debug canary mode: every guard still holds its pattern
+        const cudaError_t e = launch_guard_check(arena_, d_guard_offs_, guard_count(), status_, stream);
+        if (e != cudaSuccess) {
+            err = std::string("guard check launch failed: ") + cudaGetErrorString(e);
+            return MUON_ERR_CUDA;
+        }
+        if (launch_counter) ++*launch_counter;
     }
     return MUON_OK;
 }

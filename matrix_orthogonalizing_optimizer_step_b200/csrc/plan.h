@@ -57,6 +57,7 @@ struct LaunchRec {
     ScaleLaunch sc{};
     double flops = 0, bytes = 0;
     double extra_bytes = 0;  // the AdamW lane of a hybrid step (momentum launch)
+    char label[32] = {};     // NVTX range name of the launch (phase and chain slot)
 };
 
 struct ProfileSink {
@@ -83,6 +84,9 @@ class Plan {
     int run(cudaStream_t stream, ProfileSink* prof, long long* launch_counter, std::string& err);
     void release();
     ~Plan() { release(); }
+    // Debug canary mode: the workspace guards (none when the mode is off).
+    int guard_count() const { return static_cast<int>(guard_offs_.size()); }
+    void* guard_addr(int i) const { return static_cast<char*>(arena_) + guard_offs_[static_cast<size_t>(i)]; }
 
     std::vector<LaunchRec> launches;
     size_t arena_bytes = 0;
@@ -92,6 +96,11 @@ class Plan {
     std::vector<long long> key_;
     void* arena_ = nullptr;
     bool fault_launch_ = false;  // MUON_FAULT=launch: run() fails before its first launch
+    // MUON_DEBUG_CANARY=1: offsets of the guard after every workspace region,
+    // their device copy, and the status word the check reports to
+    std::vector<unsigned long long> guard_offs_;
+    const unsigned long long* d_guard_offs_ = nullptr;
+    DeviceStatus* status_ = nullptr;
 };
 
 // Exposed for tests of the host logic: algorithmic FLOPs of one matrix.

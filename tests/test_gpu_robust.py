@@ -32,12 +32,12 @@ SHAPES = [(256, 768), (768, 256), (200, 200), (136, 520)]
 @pytest.fixture(autouse=True)
 def _fresh(monkeypatch):
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
-    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES"):
+    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES", "MUON_DEBUG_CANARY"):
         monkeypatch.delenv(k, raising=False)
     mo.muon_reset_config()
     mo.muon_release_workspace()
     yield
-    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES"):
+    for k in ("MUON_FAULT", "MUON_WAIT_LIMIT_MS", "MUON_CHAIN_LAUNCH", "MUON_SLOT_LAUNCHES", "MUON_DEBUG_CANARY"):
         monkeypatch.delenv(k, raising=False)
     mo.muon_release_workspace()
     st, bad = mo.muon_device_status()
@@ -237,3 +237,65 @@ def test_capture_that_needs_a_plan_is_refused():
     mo.muon_step(W, G, M, lr=0.02)
     torch.cuda.synchronize()
     assert not torch.equal(W[0], W0)
+
+
+def _canary_workload():
+    """Steps over mixed, ragged and transposed shapes, a ragged orthogonalise
+    with an unaligned row pitch, and the fp32 check path; returns every output."""
+    shapes = [(768, 2304), (768, 768), (3072, 768), (200, 712), (37, 91), (136, 520), (520, 136)]
+    G = [wl.make_single(r, c, 800 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, 820 + i, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, 840 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    for _ in range(2):
+        mo.muon_step(W, G, M, lr=0.02)
+    X = torch.stack([wl.make_single(200, 333, 860 + j, "gaussian", DEV, "bf16") for j in range(3)])
+    mo.muon_orthogonalize(X, steps=5, mode="gram")
+    F = torch.stack([wl.make_single(100, 260, 870 + j, "gaussian", DEV, "f32") for j in range(2)])
+    mo.muon_orthogonalize(F, steps=5, mode="standard", fp32=True)
+    torch.cuda.synchronize()
+    return [t.clone() for t in W + M + [X, F]]
+
+
+@pytest.mark.parametrize("env", [{}, {"MUON_SLOT_LAUNCHES": "1"}])
+def test_canary_guards_stay_intact(env, monkeypatch):
+    """Debug canary mode: every workspace region followed by a guard, checked
+    after each call.  Over mixed, ragged, transposed and unaligned shapes and
+    the fp32 check path no guard is touched, and the results are bitwise
+    those of the normal layout."""
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    mo.muon_release_workspace()
+    ref = _canary_workload()
+    monkeypatch.setenv("MUON_DEBUG_CANARY", "1")
+    mo.muon_release_workspace()
+    got = _canary_workload()
+    st, _ = mo.muon_device_status()
+    assert st == mo.MUON_OK, mo.STATUS_NAMES.get(st)
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+    mo.muon_release_workspace()
+
+
+def test_canary_check_reports_an_overwritten_guard(monkeypatch):
+    """A guard overwritten between calls (a plain memset into the library's
+    own allocation, no fault) is reported by the next call's check as
+    MUON_ERR_GUARD and re-armed: the call after that is clean again."""
+    monkeypatch.setenv("MUON_DEBUG_CANARY", "1")
+    mo.muon_release_workspace()
+    shapes = [(256, 768), (200, 200)]
+    G = [wl.make_single(r, c, 900 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    W = [wl.make_single(r, c, 910 + i, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+    M = [wl.make_single(r, c, 920 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+    mo.muon_step(W, G, M, lr=0.02)
+    assert mo.muon_device_status()[0] == mo.MUON_OK
+    with pytest.raises(mo.MuonError):
+        mo.muon_debug_corrupt_guard(10 ** 6)  # no such guard
+    mo.muon_debug_corrupt_guard(3)
+    mo.muon_step(W, G, M, lr=0.02)
+    assert mo.muon_device_status()[0] == mo.MUON_ERR_GUARD
+    mo.muon_step(W, G, M, lr=0.02)
+    assert mo.muon_device_status()[0] == mo.MUON_OK
+    monkeypatch.delenv("MUON_DEBUG_CANARY")
+    mo.muon_release_workspace()
+    with pytest.raises(mo.MuonError):
+        mo.muon_debug_corrupt_guard(0)  # the mode is off: no guards

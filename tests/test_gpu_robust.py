@@ -169,12 +169,12 @@ def test_calls_alternating_streams():
             with torch.cuda.stream(streams[k % 2]):
                 mo.muon_orthogonalize(x, steps=5, mode="gram")
         if rnd == 0:
-            # round 0 equals the serial reference
+            # pass 0 equals the serial reference
             torch.cuda.synchronize()
             for a, b in zip(got, ref):
                 assert torch.equal(a, b)
     torch.cuda.synchronize()
-    # round 1 orthogonalised the outputs again: compare with the same on one stream
+    # pass 1 orthogonalised the outputs again: compare with the same on one stream
     for x in ref:
         mo.muon_orthogonalize(x, steps=5, mode="gram")
     torch.cuda.synchronize()

@@ -190,3 +190,39 @@ def test_offload_reports_bad_matrix_in_caller_numbering():
     for i in range(len(SHAPES)):
         assert torch.equal(host_p[i], Wr[i].cpu()), i
     assert torch.equal(M[7].float().isnan(), Mr[7].float().isnan())
+
+
+def test_offload_with_shape_schedules_and_soft_threshold():
+    """The offload step under a non-default config: a registered per-shape
+    schedule (4 steps), the soft-threshold split and fp32 momentum.  Every
+    group runs the same plan logic as one muon_step, so the results equal a
+    plain muon_step's bit for bit."""
+    mo.muon_set_config(soft_threshold=0.05, momentum_dtype=mo.MUON_DTYPE_F32)
+    sched = [(3.0, -3.2, 1.2), (2.8, -3.0, 1.1), (2.5, -2.6, 1.0), (2.0, -1.5, 0.5)]
+    mo.muon_set_shape_coeffs(256, 768, sched)
+    W, G, M = _make_set(SHAPES, 4700, mom_dt="f32")
+    Wr, Mr = _clone(W), _clone(M)
+    mo.muon_step(Wr, G, Mr, lr=0.1)
+    host_g = [g.cpu().pin_memory() for g in G]
+    host_p = _pinned_like(W)
+    Gd = [torch.zeros_like(g) for g in G]
+    mo.muon_step_offload(W, Gd, M, grads_host=host_g, params_host=host_p, lr=0.1, chunks=4)
+    torch.cuda.synchronize()
+    _check_equal(W, M, Wr, Mr, host_p)
+
+
+def test_offload_under_canary_guards(monkeypatch):
+    """Debug canary mode over the offload step: every group's plan keeps its
+    guards intact, and the results are those of the normal layout."""
+    W, G, M = _make_set(SHAPES, 4800)
+    Wr, Mr = _clone(W), _clone(M)
+    host_g = [g.cpu().pin_memory() for g in G]
+    Gd = [torch.zeros_like(g) for g in G]
+    mo.muon_step_offload(Wr, Gd, Mr, grads_host=host_g, lr=0.1, chunks=3)
+    monkeypatch.setenv("MUON_DEBUG_CANARY", "1")
+    mo.muon_release_workspace()
+    mo.muon_step_offload(W, Gd, M, grads_host=host_g, lr=0.1, chunks=3)
+    assert mo.muon_device_status()[0] == mo.MUON_OK
+    monkeypatch.delenv("MUON_DEBUG_CANARY")
+    mo.muon_release_workspace()
+    _check_equal(W, M, Wr, Mr)

@@ -299,3 +299,53 @@ def test_canary_check_reports_an_overwritten_guard(monkeypatch):
     mo.muon_release_workspace()
     with pytest.raises(mo.MuonError):
         mo.muon_debug_corrupt_guard(0)  # the mode is off: no guards
+
+
+def test_orthogonalize_captured_in_a_cuda_graph():
+    """muon_orthogonalize captured after one eager call (its plan exists) and
+    replayed twice equals three eager calls bit for bit."""
+    X = torch.stack([wl.make_single(512, 1536, 940 + j, "gaussian", DEV, "bf16") for j in range(3)])
+    Xr = X.clone()
+    for _ in range(3):
+        mo.muon_orthogonalize(Xr, steps=5, mode="gram")
+    mo.muon_orthogonalize(X, steps=5, mode="gram")
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        mo.muon_orthogonalize(X, steps=5, mode="gram")
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(X, Xr)
+    del graph
+    mo.muon_release_workspace()
+
+
+def test_hybrid_step_under_canary_guards(monkeypatch):
+    """Debug canary mode over the hybrid step (the AdamW lane in the momentum
+    launch's grid): guards intact, results equal to the normal layout."""
+    shapes = [(256, 768), (200, 200), (37, 91)]
+    numels = [50257 * 8, 768, 7]
+
+    def run():
+        W = [wl.make_single(r, c, 960 + i, "params", DEV, "f32") for i, (r, c) in enumerate(shapes)]
+        G = [wl.make_single(r, c, 970 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+        M = [wl.make_single(r, c, 980 + i, "student_t3", DEV, "bf16", 0.01) for i, (r, c) in enumerate(shapes)]
+        P = [wl.make_single(1, n, 990 + i, "params", DEV, "f32").view(-1) for i, n in enumerate(numels)]
+        AG = [wl.make_single(1, n, 995 + i, "student_t3", DEV, "bf16", 0.01).view(-1) for i, n in enumerate(numels)]
+        M1 = [torch.zeros(n, device=DEV) for n in numels]
+        M2 = [torch.zeros(n, device=DEV) for n in numels]
+        for t in (1, 2):
+            mo.muon_hybrid_step(W, G, M, P, AG, M1, M2, t)
+        torch.cuda.synchronize()
+        return [x.clone() for x in W + M + P + M1 + M2]
+
+    ref = run()
+    monkeypatch.setenv("MUON_DEBUG_CANARY", "1")
+    mo.muon_release_workspace()
+    got = run()
+    assert mo.muon_device_status()[0] == mo.MUON_OK
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
+    monkeypatch.delenv("MUON_DEBUG_CANARY")
+    mo.muon_release_workspace()

@@ -77,6 +77,18 @@ constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BNH * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
+// Tile width: NT halves of 256 columns.  NT = 2 (persistent launches of long-K
+// products): a CTA pair computes a 256 x 512 tile, both N halves from the
+// same A slice, so a quarter fewer operand bytes per FLOP; the one 512-column
+// accumulator takes all of TMEM (the epilogue no longer overlaps the next
+// tile's main loop) and 4 stages of 48 KB fit.
+template <int NT>
+__host__ __device__ constexpr int stages_of() { return NT == 1 ? STAGES : 4; }
+template <int NT>
+__host__ __device__ constexpr int stage_bytes_of() { return A_BYTES + NT * B_BYTES; }
+template <int NT>
+__host__ __device__ constexpr int num_acc_of() { return NT == 1 ? 2 : 1; }  // TMEM accumulators (512 columns in all)
+
 constexpr int EPI_WARPS = 8;
 constexpr int SCHED_WARP = 2 + EPI_WARPS;       // the tile scheduler (after the epilogue warps)
 constexpr int NUM_THREADS = 96 + 32 * EPI_WARPS;
@@ -87,23 +99,30 @@ constexpr int STORE_BYTES = EPI_WARPS * 2 * STORE_BOX_BYTES;  // two boxes per e
 constexpr int SCHED = 4;  // depth of the tile-record ring: the scheduler's lookahead
 // The epilogue warps as GROUPS groups (1 or 2), each taking every GROUPS-th
 // tile of the pair.
-template <int GROUPS>
+template <int GROUPS, int NT = 1>
 struct EpiShape {
     static constexpr int group_warps = EPI_WARPS / GROUPS;
-    static constexpr int cols = BN / (group_warps / 4);  // tile columns per epilogue warp
+    static constexpr int cols = BN * NT / (group_warps / 4);  // tile columns per epilogue warp
     // readers of every ring slot: in the leader its producer, its MMA thread
     // and the epilogue warps of the group that takes the tile; in the peer
     // its producer and that group's epilogue warps
     static constexpr uint32_t readers_leader = 2 + group_warps;
     static constexpr uint32_t readers_peer = 1 + group_warps;
     static_assert(group_warps % 4 == 0, "a group covers the four TMEM lane quarters");
-    static_assert(2 % GROUPS == 0 && SCHED % GROUPS == 0, "a group owns whole accumulators and ring slots");
+    static_assert(num_acc_of<NT>() % GROUPS == 0 && SCHED % GROUPS == 0,
+                  "a group owns whole accumulators and ring slots");
 };
 constexpr int kChainGroups = 2;  // epilogue groups of a chained launch (persistent launches: 1)
 static_assert(kTileArrivals == 2 * EpiShape<kChainGroups>::group_warps,
               "chain completions are counted per tile: one group's warps in each CTA");
 constexpr size_t SMEM_BYTES = STAGES * STAGE_BYTES + STORE_BYTES + 1024 /*align slack*/ + 1024 /*barriers, ring*/;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a CTA may use");
+template <int NT>
+constexpr size_t smem_bytes() {
+    return static_cast<size_t>(stages_of<NT>()) * stage_bytes_of<NT>() + STORE_BYTES + 1024 + 1024;
+}
+static_assert(smem_bytes<2>() <= 232448, "over the 227 KB of shared memory a CTA may use");
+static_assert(stages_of<2>() <= STAGES, "barrier arrays");
 
 // A ring slot: the raw 32-byte tile record (TcTile), or kRingEnd in its
 // first word once the launch's tiles are exhausted.
@@ -224,7 +243,9 @@ struct RingReader {
 
 __device__ __forceinline__ RingRec end_rec() { return RingRec{make_uint4(kRingEnd, 0, 0, 0), make_uint4(0, 0, 0, 0)}; }
 
+template <int NT>
 __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t rank) {
+    constexpr int kStages = stages_of<NT>(), kStageBytes = stage_bytes_of<NT>();
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
     const bool leader = rank == 0;
@@ -280,21 +301,18 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
             last_b = tile.b_map;
         }
         const int arow = bi * BMP + static_cast<int>(rank) * BM;   // this CTA's A rows
-        const int brow = bj * BN + static_cast<int>(rank) * BNH;   // this CTA's B rows (N)
         const int nk = (K + BK - 1) / BK;
         for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait(&sh->empty[stage], phase ^ 1u, abort_flag, lim)) {
                 ok = false;
                 break;
             }
-            uint8_t* sa = tiles_smem + stage * STAGE_BYTES;
-            uint8_t* sb = sa + A_BYTES;
+            uint8_t* sa = tiles_smem + stage * kStageBytes;
             const uint32_t full_leader = map_to_cta(smem_u32(&sh->full[stage]), 0);
-            if (leader) mbar_arrive_expect_tx(&sh->full[stage], 2 * STAGE_BYTES);
+            if (leader) mbar_arrive_expect_tx(&sh->full[stage], 2 * kStageBytes);
             // a K slice of a symmetric operand below its stored upper tiles is
             // read transposed from the mirrored tile (same values)
             const bool a_t = a_mn || (a_sym && slice_is_lower(bi, kb));
-            const bool b_t = b_mn || (b_sym && slice_is_lower(bj, kb));
             if (!a_t) {
                 tma_load_3d_pair(sa, ma, full_leader, kb * BK, arow, a_z);
             } else {
@@ -302,15 +320,23 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
                 for (int j = 0; j < BM / 64; ++j)
                     tma_load_3d_pair(sa + j * MN_BLOCK_BYTES, ma_t, full_leader, arow + 64 * j, kb * BK, a_z);
             }
-            if (!b_t) {
-                tma_load_3d_pair(sb, mb, full_leader, kb * BK, brow, b_z);
-            } else {
 #pragma unroll
-                for (int j = 0; j < BNH / 64; ++j)
-                    tma_load_3d_pair(sb + j * MN_BLOCK_BYTES, mb_t, full_leader, brow + 64 * j, kb * BK, b_z);
+            for (int h = 0; h < NT; ++h) {
+                // N half h: 256-column block bj * NT + h, this CTA's 128 rows of it
+                const int blk = bj * NT + h;
+                const int brow = blk * BN + static_cast<int>(rank) * BNH;
+                uint8_t* sb = sa + A_BYTES + h * B_BYTES;
+                const bool b_t = b_mn || (b_sym && slice_is_lower(blk, kb));
+                if (!b_t) {
+                    tma_load_3d_pair(sb, mb, full_leader, kb * BK, brow, b_z);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < BNH / 64; ++j)
+                        tma_load_3d_pair(sb + j * MN_BLOCK_BYTES, mb_t, full_leader, brow + 64 * j, kb * BK, b_z);
+                }
             }
             ++issued;
-            if (++stage == STAGES) {
+            if (++stage == kStages) {
                 stage = 0;
                 phase ^= 1u;
             }
@@ -337,10 +363,10 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
     // Drain (leader): the last fills of every stage must have landed before
     // the pair exits.  Fill i used stage i % STAGES, phase parity (i / STAGES) & 1.
     if (leader) {
-        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+        const uint32_t first = issued > kStages ? issued - kStages : 0;
         int never = 0;
         for (uint32_t i = first; i < issued; ++i) {
-            if (!mbar_wait(&sh->full[i % STAGES], (i / STAGES) & 1u, &never, lim)) {
+            if (!mbar_wait(&sh->full[i % kStages], (i / kStages) & 1u, &never, lim)) {
                 atomicOr(&L.status->bits, ST_TIMEOUT);
                 break;
             }
@@ -370,7 +396,9 @@ __device__ void scheduler(const TcLaunch& L, Shared* sh) {
     }
 }
 
+template <int NT>
 __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uint32_t tmem_base) {
+    constexpr int kStages = stages_of<NT>(), kStageBytes = stage_bytes_of<NT>(), kAcc = num_acc_of<NT>();
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
     int stage = 0;
@@ -401,38 +429,42 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN * NT);
         for (int kb = 0; kb < nk; ++kb) {
             if (!mbar_wait(&sh->full[stage], phase, abort_flag, lim)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t a_addr = tiles_base + stage * STAGE_BYTES;
-            const uint32_t b_addr = a_addr + A_BYTES;
+            const uint32_t a_addr = tiles_base + stage * kStageBytes;
             const int a_t = (a_mn || (a_sym && slice_is_lower(bi, kb))) ? 1 : 0;  // as loaded by the producer
-            const int b_t = (b_mn || (b_sym && slice_is_lower(bj, kb))) ? 1 : 0;
-            const uint32_t idesc = make_instr_desc(fmt, a_t, b_t, BMP, BN);
 #pragma unroll
-            for (int k = 0; k < BK / 16; ++k) {
-                // K-major: advance 16 elements (32 B) inside the swizzled row;
-                // MN-major: advance 16 k-rows (two 8-row groups of 1024 B).
-                const uint64_t ad = a_t ? make_smem_desc(a_addr + k * 2048, MN_BLOCK_BYTES, 1024)
-                                        : make_smem_desc(a_addr + k * 32, 16, 1024);
-                const uint64_t bd = b_t ? make_smem_desc(b_addr + k * 2048, MN_BLOCK_BYTES, 1024)
-                                        : make_smem_desc(b_addr + k * 32, 16, 1024);
-                umma_f16_pair(d_tmem, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+            for (int h = 0; h < NT; ++h) {
+                // N half h: its own B slice, accumulator columns [256 h, 256 h + 256)
+                const uint32_t b_addr = a_addr + A_BYTES + h * B_BYTES;
+                const int b_t = (b_mn || (b_sym && slice_is_lower(bj * NT + h, kb))) ? 1 : 0;
+                const uint32_t idesc = make_instr_desc(fmt, a_t, b_t, BMP, BN);
+#pragma unroll
+                for (int k = 0; k < BK / 16; ++k) {
+                    // K-major: advance 16 elements (32 B) inside the swizzled row;
+                    // MN-major: advance 16 k-rows (two 8-row groups of 1024 B).
+                    const uint64_t ad = a_t ? make_smem_desc(a_addr + k * 2048, MN_BLOCK_BYTES, 1024)
+                                            : make_smem_desc(a_addr + k * 32, 16, 1024);
+                    const uint64_t bd = b_t ? make_smem_desc(b_addr + k * 2048, MN_BLOCK_BYTES, 1024)
+                                            : make_smem_desc(b_addr + k * 32, 16, 1024);
+                    umma_f16_pair(d_tmem + static_cast<uint32_t>(h * BN), ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                }
             }
             issued_any = true;
             umma_commit_pair(&sh->empty[stage], 0x3);  // both CTAs may refill this slot
-            if (++stage == STAGES) {
+            if (++stage == kStages) {
                 stage = 0;
                 phase ^= 1u;
             }
         }
         if (!ok) break;
         umma_commit_pair(&sh->tfull[acc], 0x3);  // accumulator ready in both CTAs
-        if (++acc == 2) {
+        if (++acc == kAcc) {
             acc = 0;
             acc_phase ^= 1u;
         }
@@ -448,10 +480,11 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
     }
 }
 
-template <int GROUPS>
+template <int GROUPS, int NT>
 __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint32_t tmem_base, int warp, int lane,
                                uint32_t rank) {
-    using S = EpiShape<GROUPS>;
+    using S = EpiShape<GROUPS, NT>;
+    constexpr int kAcc = num_acc_of<NT>();
     volatile int* abort_flag = &sh->abort;
     const unsigned long long lim = L.wait_ns;
     const int q = warp & 3;                       // TMEM lane quarter this warp may access
@@ -459,8 +492,8 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     const int part = ((warp - 2) % S::group_warps) >> 2;  // column part of the tile
     const uint32_t tempty_leader[2] = {map_to_cta(smem_u32(&sh->tempty[0]), 0),
                                        map_to_cta(smem_u32(&sh->tempty[1]), 0)};
-    // tile i of the pair uses accumulator i % 2 (the MMA thread alternates)
-    int acc = group % 2;
+    // tile i of the pair uses accumulator i % kAcc (the MMA thread alternates)
+    int acc = group % kAcc;
     uint32_t acc_phase = 0;
     unsigned seen_mat = ~0u, seen_done = 0;
     uint32_t nstored = 0;  // TMA store boxes issued by this warp (alternating buffers)
@@ -499,11 +532,15 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             seen_mat = tile.mat;
             seen_done = tile.need;
         }
-        const bool skip = ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0;
+        // a 512-wide tile of a symmetric output may reach below the diagonal:
+        // a part whose 256-column block is a lower block is not stored (only
+        // upper blocks are; their consumers read lower blocks transposed)
+        const bool lower = NT > 1 && L.problems[tile.problem].pad_ != 0 && bi > bj * NT + part;
+        const bool skip = (ep.skip_idx >= 0 && L.bad[ep.skip_idx] != 0) || lower;
         const float sig = ep.sigma ? *ep.sigma : 1.f;
         const long long row0 = static_cast<long long>(bi) * BMP + rank * BM + q * 32;  // this warp's first row
         const long long row = row0 + lane;
-        const int cbase = bj * BN + part * S::cols;
+        const int cbase = bj * BN * NT + part * S::cols;
         const bool use_tma = ep.o1_map >= 0;
         const CUtensorMap* omap = use_tma ? L.maps + ep.o1_map : nullptr;
         if (use_tma && ep.o1_map != last_map) {
@@ -556,7 +593,7 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             }
             uint32_t r[32];
             __syncwarp();
-            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + part * S::cols + c, r);
+            tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN * NT + part * S::cols + c, r);
             tmem_wait_ld();
             if (skip || row0 >= PM) {  // warp-uniform
                 pre = nxt;
@@ -623,8 +660,8 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
             if (lane == 0) red_release_add_gpu(L.done + tile.mat, 1u);
         }
         acc += GROUPS;  // this group's next tile
-        if (acc >= 2) {
-            acc -= 2;
+        if (acc >= kAcc) {
+            acc -= kAcc;
             acc_phase ^= 1u;
         }
     }
@@ -634,20 +671,21 @@ __device__ void epilogue_warps(const TcLaunch& L, Shared* sh, uint32_t stg, uint
     __syncwarp();
 }
 
-template <int GROUPS>
+template <int GROUPS, int NT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ TcLaunch L) {
-    using S = EpiShape<GROUPS>;
+    using S = EpiShape<GROUPS, NT>;
+    constexpr int kStages = stages_of<NT>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* tiles_smem =
         reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint8_t* store_smem = tiles_smem + STAGES * STAGE_BYTES;  // 1024-byte aligned boxes
+    uint8_t* store_smem = tiles_smem + kStages * stage_bytes_of<NT>();  // 1024-byte aligned boxes
     Shared* sh = reinterpret_cast<Shared*>(store_smem + STORE_BYTES);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const uint32_t rank = cluster_cta_rank();
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&sh->full[s], 1);
             mbar_init(&sh->empty[s], 1);
         }
@@ -675,13 +713,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tmem_base = sh->tmem_base;
 
     if (warp == 0) {
-        if (lane == 0) producer(L, tiles_smem, sh, rank);
+        if (lane == 0) producer<NT>(L, tiles_smem, sh, rank);
     } else if (warp == 1) {
-        if (lane == 0 && rank == 0) mma_issuer(L, tiles_smem, sh, tmem_base);
+        if (lane == 0 && rank == 0) mma_issuer<NT>(L, tiles_smem, sh, tmem_base);
     } else if (warp == SCHED_WARP) {
         if (lane == 0 && rank == 0) scheduler<GROUPS>(L, sh);
     } else {
-        epilogue_warps<GROUPS>(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane, rank);
+        epilogue_warps<GROUPS, NT>(L, sh, smem_u32(store_smem + (warp - 2) * 2 * STORE_BOX_BYTES), tmem_base, warp, lane,
+                                   rank);
     }
 
     tc_fence_before();
@@ -699,17 +738,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 size_t gemm_tc_smem_bytes() { return SMEM_BYTES; }
 int gemm_tc_tile_m() { return BMP; }
 int gemm_tc_tile_n() { return BN; }
+int gemm_tc_wide_tile_n() { return 2 * BN; }
 
 namespace {
 // CTA pairs of one instance that can be resident at once.
-template <int GROUPS>
+template <int GROUPS, int NT>
 int max_pairs_of() {
-    cudaFuncSetAttribute(gemm_tc_kernel<GROUPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(SMEM_BYTES));
+    cudaFuncSetAttribute(gemm_tc_kernel<GROUPS, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem_bytes<NT>()));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem_bytes<NT>();
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
     attr.val.clusterDim.x = 2;
@@ -718,7 +758,7 @@ int max_pairs_of() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GROUPS>, &cfg) != cudaSuccess) {
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<GROUPS, NT>, &cfg) != cudaSuccess) {
         cudaGetLastError();
         n = 0;
     }
@@ -731,27 +771,33 @@ int max_pairs_of() {
 int gemm_tc_max_pairs() {
     static int cached = -1;
     if (cached >= 0) return cached;
-    cached = std::min(max_pairs_of<1>(), max_pairs_of<kChainGroups>());
+    cached = std::min(std::min(max_pairs_of<1, 1>(), max_pairs_of<kChainGroups, 1>()), max_pairs_of<1, 2>());
     return cached;
 }
 
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream) {
     static bool configured = false;
     if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(SMEM_BYTES));
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem_bytes<1>()));
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gemm_tc_kernel<kChainGroups>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(SMEM_BYTES));
+            e = cudaFuncSetAttribute(gemm_tc_kernel<kChainGroups, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_bytes<1>()));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_tc_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_bytes<2>()));
         if (e != cudaSuccess) return e;
         configured = true;
     }
     if (L.ntiles <= 0) return cudaSuccess;
-    // chained launches (chain counters) split the epilogue into two groups
+    // chained launches (chain counters) split the epilogue into two groups;
+    // persistent launches of 512-wide tiles take the wide instance
     if (L.done)
-        gemm_tc_kernel<kChainGroups><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(L);
+        gemm_tc_kernel<kChainGroups, 1><<<grid, NUM_THREADS, smem_bytes<1>(), stream>>>(L);
+    else if (L.nt == 2)
+        gemm_tc_kernel<1, 2><<<grid, NUM_THREADS, smem_bytes<2>(), stream>>>(L);
     else
-        gemm_tc_kernel<1><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(L);
+        gemm_tc_kernel<1, 1><<<grid, NUM_THREADS, smem_bytes<1>(), stream>>>(L);
     return cudaGetLastError();
 }
 

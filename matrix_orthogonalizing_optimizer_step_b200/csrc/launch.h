@@ -44,6 +44,7 @@ struct TcLaunch {
     unsigned* ticket;     // next unclaimed tile (zeroed before the launch)
     unsigned long long wait_ns;  // bound of every wait of the launch
     DeviceStatus* status;
+    int nt;               // tile width in 256-column halves (1, or 2 for persistent launches)
 };
 
 constexpr unsigned kTileArrivals = 8;  // epilogue warps of a CTA pair that take one tile (one group per CTA)
@@ -51,6 +52,7 @@ constexpr unsigned kTileArrivals = 8;  // epilogue warps of a CTA pair that take
 size_t gemm_tc_smem_bytes();
 int gemm_tc_tile_m();
 int gemm_tc_tile_n();
+int gemm_tc_wide_tile_n();  // 512: the tile width of the wide (NT = 2) instance
 int gemm_tc_max_pairs();
 cudaError_t launch_gemm_tc(const TcLaunch& L, int grid, cudaStream_t stream);
 

@@ -59,7 +59,7 @@ struct TcProblem {
     int a_mn, b_mn;        // 1: operand is MN-major in memory
     int a_sym, b_sym;      // 1: operand is an upper-stored symmetric matrix
     int fmt;               // 0 = f16 operands, 1 = bf16 operands
-    int pad_;
+    int pad_;              // 1: the output is symmetric (upper 256-blocks are stored)
     Epilogue ep;
 };
 

@@ -85,6 +85,13 @@ int fault_mode() {
     return FAULT_NONE;
 }
 
+// MUON_TILE_N=256 (read when a plan is built): persistent launches keep
+// 256-wide tiles instead of 512-wide ones.
+bool wide_tiles_allowed() {
+    const char* v = std::getenv("MUON_TILE_N");
+    return !(v && std::atoi(v) == 256);
+}
+
 bool canary_mode() {
     const char* v = std::getenv("MUON_DEBUG_CANARY");
     return v && v[0] == '1';
@@ -379,6 +386,7 @@ static std::vector<long long> make_key(const PlanRequest& rq) {
     for (int si : rq.sched) k.push_back(si);
     k.push_back(fault_mode());
     k.push_back(canary_mode() ? 1 : 0);
+    k.push_back(wide_tiles_allowed() ? 1 : 0);
     k.push_back(static_cast<long long>(wait_limit_ns()));
     for (size_t i = 0; i < rq.rows.size(); ++i) {
         k.push_back(rq.rows[i]);
@@ -638,6 +646,25 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         if (std::getenv("MUON_SLOT_LAUNCHES")) chained = false;
         if (fault == FAULT_TIMEOUT) chained = true;  // the injected wait is a chain dependency
     }
+    // Persistent (per-slot) launches of long products use 256 x 512 tiles: a
+    // quarter fewer operand bytes per FLOP, but one accumulator (the epilogue
+    // no longer overlaps the next tile's main loop), and on symmetric outputs
+    // more tile area computed below the diagonal.  A launch takes them when
+    // its FLOP-weighted K is at least kWideMinK (shorter, the exposed epilogue
+    // costs more than the bytes save) and its wide tiles compute at most
+    // kWideMaxArea times the area of its 256-wide ones, K-weighted (n = 4096
+    // symmetric products: 1.06; n = 2048: 1.11).  Chained launches keep
+    // 256 x 256 tiles and the double-buffered accumulators.
+    constexpr double kWideMinK = 3072.0, kWideMaxArea = 1.08;
+    const bool wide = !f32 && !chained && wide_tiles_allowed();
+    // 256 x tw tiles of an M x N output (symmetric: those not wholly below the diagonal)
+    auto tile_count = [&](int M, int N, int tw, bool sym) {
+        long long n = 0;
+        for (int bi = 0; bi < (M + tile_m - 1) / tile_m; ++bi)
+            for (int bj = 0; bj < (N + tw - 1) / tw; ++bj)
+                if (!(sym && bi * tile_m > bj * tw + tw - 1)) ++n;
+        return n;
+    };
     const unsigned long long wait_ns = wait_limit_ns();
     size_t nticket = 0;  // tickets handed out so far (one per GEMM launch)
     auto buf_ptr = [&](const Group& g, int b, int z) -> char* {
@@ -838,9 +865,30 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     };
 
     for (size_t si = 0; si < nslots; ++si) {
+        bool slot_wide = false;
+        if (wide) {
+            double fk = 0.0, fsum = 0.0, area_w = 0.0, area_n = 0.0;
+            for (const Group& g : groups) {
+                if (si >= g.slots.size()) continue;
+                for (const OpDesc& op : g.slots[si]) {
+                    int M, N, K;
+                    OperandGeom A, B;
+                    op_geometry(g, op, M, N, K, A, B);
+                    const double f = op_flops(g, op) * static_cast<double>(g.mats.size());
+                    fk += f * K;
+                    fsum += f;
+                    const double kw = static_cast<double>(K) * static_cast<double>(g.mats.size());
+                    area_n += kw * static_cast<double>(tile_count(M, N, tile_n, op.sym));
+                    area_w += 2.0 * kw * static_cast<double>(tile_count(M, N, gemm_tc_wide_tile_n(), op.sym));
+                }
+            }
+            slot_wide = fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n;
+        }
+        const int slot_tile_n = slot_wide ? gemm_tc_wide_tile_n() : tile_n;
         LaunchRec lr;
         lr.kind = f32 ? LaunchRec::F32 : LaunchRec::TC;
-        std::snprintf(lr.label, sizeof(lr.label), f32 ? "muon gemm_f32 slot %zu" : "muon gemm slot %zu", si);
+        std::snprintf(lr.label, sizeof(lr.label), f32 ? "muon gemm_f32 slot %zu" : "muon gemm slot %zu x%d", si,
+                      slot_tile_n);
         const size_t prob_begin = f32 ? fprobs.size() : tprobs.size();
         const size_t tile_begin = tiles.size();
         struct TileRef {
@@ -945,11 +993,13 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                         p.a_mn = A.mn ? 1 : 0;
                         p.b_mn = B.mn ? 1 : 0;
                         p.fmt = g.dt[A.buf] == DT_F16 ? 0 : 1;
+                        p.pad_ = op.sym ? 1 : 0;  // symmetric output: only its upper 256-blocks are stored
                         p.ep = ep;
                         p.ep.sym = 0;  // upper tiles only (tile list below), no mirrored stores
                         const unsigned pi = static_cast<unsigned>(tprobs.size());
                         tprobs.push_back(p);
-                        const int tm = (M + tile_m - 1) / tile_m, tn = (N + tile_n - 1) / tile_n;
+                        const int tw = slot_tile_n;  // tile width of this launch
+                        const int tm = (M + tile_m - 1) / tile_m, tn = (N + tw - 1) / tw;
                         // Tile order within a problem: consecutive tiles (the ones
                         // the pairs work on at once) should share the panels of
                         // the big operand.  A non-transposed apply (n x n factor
@@ -961,7 +1011,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                         for (int o = 0; o < outer; ++o)
                             for (int i2 = 0; i2 < inner; ++i2) {
                                 const int bi = col_major ? i2 : o, bj = col_major ? o : i2;
-                                if (op.sym && bi * tile_m > bj * tile_n + tile_n - 1) continue;
+                                if (op.sym && bi * tile_m > bj * tw + tw - 1) continue;  // wholly below the diagonal
                                 TcTile tt;
                                 std::memset(&tt, 0, sizeof(tt));
                                 tt.problem = pi;
@@ -1024,6 +1074,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
             lr.tc.ticket = d_done + nm + nticket++;
             lr.tc.wait_ns = wait_ns;
             lr.tc.status = status;
+            lr.tc.nt = slot_wide ? 2 : 1;
             // CTA pairs: one cluster of 2 per tile, at most one CTA per SM
             lr.grid = 2 * std::max(1, std::min(lr.tc.ntiles, num_sms / 2));
         }
@@ -1040,6 +1091,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
         chain.tc.ticket = d_done + nm + nticket++;
         chain.tc.wait_ns = wait_ns;
         chain.tc.status = status;
+        chain.tc.nt = 1;
         // one pair per co-resident cluster slot; tiles are claimed in list
         // order, so pairs that are not resident at once delay nothing
         chain.grid = 2 * std::max(1, std::min(chain.tc.ntiles, max_pairs));

@@ -9,14 +9,18 @@
 // issues M=256 N=256 K=16 MMAs that read both CTAs' shared memory, and each
 // CTA's TMEM receives its 128 rows of the fp32 accumulator.  Per CTA and
 // 64-wide K slice this moves 32 KB of operands for 4.2 MFLOP, a third less
-// than a single-CTA 128 x 256 tile.
+// than a single-CTA 128 x 256 tile.  Persistent launches of long products use
+// 256 x 512 tiles instead (the NT = 2 instance): two N=256 MMAs on the same A
+// slice into one 512-column accumulator, 48 KB per CTA and K slice for
+// 8.4 MFLOP.
 //
 //   warp 10     tile scheduler (leader CTA): claims tiles, publishes records
 //   warp 0      TMA producer (both CTAs): 64-wide K slices of its halves of A
 //               and B into a 5-stage ring (128-byte swizzle, no multicast);
 //               the transaction bytes of both CTAs land on the leader's barrier
 //   warp 1      TMEM owner (both CTAs) and MMA issuer (leader only):
-//               two 256-column fp32 accumulators (double-buffered)
+//               two 256-column fp32 accumulators (double-buffered), or one of
+//               512 columns for 256 x 512 tiles
 //   warps 2..9  epilogue: tcgen05.ld of 32-column slices of the warp's TMEM
 //               lane quarter (32 rows), fused combine
 //               sigma*(alpha*acc + beta*C1) + gamma*C2 + delta*I; each warp

@@ -290,6 +290,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
         const bool a_mn = fl & TILE_A_MN, b_mn = fl & TILE_B_MN, a_sym = fl & TILE_A_SYM, b_sym = fl & TILE_B_SYM;
         const int a_z = tile.a_z, b_z = tile.b_z;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
+        const int h0 = (NT > 1 && (fl & TILE_LOWER0)) ? 1 : 0;  // first N half skipped (lower block)
         const CUtensorMap* ma = L.maps + tile.a_map;
         const CUtensorMap* mb = L.maps + tile.b_map;
         const CUtensorMap* ma_t = a_sym ? L.maps + tile.a_map_t : ma;
@@ -313,7 +314,8 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
             }
             uint8_t* sa = tiles_smem + stage * kStageBytes;
             const uint32_t full_leader = map_to_cta(smem_u32(&sh->full[stage]), 0);
-            if (leader) mbar_arrive_expect_tx(&sh->full[stage], 2 * kStageBytes);
+            // both CTAs' A slice and the B halves this tile computes
+            if (leader) mbar_arrive_expect_tx(&sh->full[stage], 2 * (A_BYTES + (NT - h0) * B_BYTES));
             // a K slice of a symmetric operand below its stored upper tiles is
             // read transposed from the mirrored tile (same values)
             const bool a_t = a_mn || (a_sym && slice_is_lower(bi, kb));
@@ -326,6 +328,7 @@ __device__ void producer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, uin
             }
 #pragma unroll
             for (int h = 0; h < NT; ++h) {
+                if (h < h0) continue;
                 // N half h: 256-column block bj * NT + h, this CTA's 128 rows of it
                 const int blk = bj * NT + h;
                 const int brow = blk * BN + static_cast<int>(rank) * BNH;
@@ -427,6 +430,7 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
         const int a_sym = (fl & TILE_A_SYM) ? 1 : 0, b_sym = (fl & TILE_B_SYM) ? 1 : 0;
         const int fmt = (fl & TILE_BF16) ? 1 : 0;
         const int bi = static_cast<int>(tile.bibj >> 16), bj = static_cast<int>(tile.bibj & 0xFFFFu);
+        const int h0 = (NT > 1 && (fl & TILE_LOWER0)) ? 1 : 0;  // first N half skipped (lower block)
         const int nk = (K + BK - 1) / BK;
         if (!mbar_wait(&sh->tempty[acc], acc_phase ^ 1u, abort_flag, lim)) {
             ok = false;
@@ -444,6 +448,7 @@ __device__ void mma_issuer(const TcLaunch& L, uint8_t* tiles_smem, Shared* sh, u
             const int a_t = (a_mn || (a_sym && slice_is_lower(bi, kb))) ? 1 : 0;  // as loaded by the producer
 #pragma unroll
             for (int h = 0; h < NT; ++h) {
+                if (h < h0) continue;
                 // N half h: its own B slice, accumulator columns [256 h, 256 h + 256)
                 const uint32_t b_addr = a_addr + A_BYTES + h * B_BYTES;
                 const int b_t = (b_mn || (b_sym && slice_is_lower(bj * NT + h, kb))) ? 1 : 0;

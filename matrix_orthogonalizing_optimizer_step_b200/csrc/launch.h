@@ -26,7 +26,9 @@ struct TcTile {
     unsigned short a_z, b_z;                          // batch coordinates
 };
 static_assert(sizeof(TcTile) == 32, "tile records are loaded as two 16-byte vectors");
-enum { TILE_A_MN = 1, TILE_B_MN = 2, TILE_A_SYM = 4, TILE_B_SYM = 8, TILE_BF16 = 16 };
+// TILE_LOWER0: a 256 x 512 tile of a symmetric output whose first 256-column
+// half is a lower block: that half is neither loaded, computed nor stored.
+enum { TILE_A_MN = 1, TILE_B_MN = 2, TILE_A_SYM = 4, TILE_B_SYM = 8, TILE_BF16 = 16, TILE_LOWER0 = 32 };
 constexpr unsigned kTileMaxK = (1u << 24) - 1;
 
 // Tiles are claimed in list order from `ticket` (a global counter, zero at

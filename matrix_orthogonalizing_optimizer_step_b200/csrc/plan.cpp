@@ -649,20 +649,26 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     // Persistent (per-slot) launches of long products use 256 x 512 tiles: a
     // quarter fewer operand bytes per FLOP, but one accumulator (the epilogue
     // no longer overlaps the next tile's main loop), and on symmetric outputs
-    // more tile area computed below the diagonal.  A launch takes them when
-    // its FLOP-weighted K is at least kWideMinK (shorter, the exposed epilogue
-    // costs more than the bytes save) and its wide tiles compute at most
-    // kWideMaxArea times the area of its 256-wide ones, K-weighted (n = 4096
-    // symmetric products: 1.06; n = 2048: 1.11).  Chained launches keep
-    // 256 x 256 tiles and the double-buffered accumulators.
+    // more tile area computed below the diagonal of symmetric outputs (a wide
+    // tile whose first half is a lower block skips that half: TILE_LOWER0).
+    // A launch takes them when its FLOP-weighted K is at least kWideMinK
+    // (shorter, the exposed epilogue costs more than the bytes save) and its
+    // wide tiles compute at most kWideMaxArea times the area of its 256-wide
+    // ones, K-weighted.  Chained launches keep 256 x 256 tiles and the
+    // double-buffered accumulators.
     constexpr double kWideMinK = 3072.0, kWideMaxArea = 1.08;
     const bool wide = !f32 && !chained && wide_tiles_allowed();
-    // 256 x tw tiles of an M x N output (symmetric: those not wholly below the diagonal)
-    auto tile_count = [&](int M, int N, int tw, bool sym) {
+    // 256-column blocks computed by the 256 x tw tiles of an M x N output
+    // (symmetric: tiles wholly below the diagonal are left out, and a wide
+    // tile's lower first half is not computed)
+    auto block_count = [&](int M, int N, int tw, bool sym) {
+        const int per = tw / tile_n;
         long long n = 0;
         for (int bi = 0; bi < (M + tile_m - 1) / tile_m; ++bi)
-            for (int bj = 0; bj < (N + tw - 1) / tw; ++bj)
-                if (!(sym && bi * tile_m > bj * tw + tw - 1)) ++n;
+            for (int bj = 0; bj < (N + tw - 1) / tw; ++bj) {
+                if (sym && bi * tile_m > bj * tw + tw - 1) continue;
+                n += (sym && per > 1 && bi > bj * per) ? per - 1 : per;
+            }
         return n;
     };
     const unsigned long long wait_ns = wait_limit_ns();
@@ -878,8 +884,8 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                     fk += f * K;
                     fsum += f;
                     const double kw = static_cast<double>(K) * static_cast<double>(g.mats.size());
-                    area_n += kw * static_cast<double>(tile_count(M, N, tile_n, op.sym));
-                    area_w += 2.0 * kw * static_cast<double>(tile_count(M, N, gemm_tc_wide_tile_n(), op.sym));
+                    area_n += kw * static_cast<double>(block_count(M, N, tile_n, op.sym));
+                    area_w += kw * static_cast<double>(block_count(M, N, gemm_tc_wide_tile_n(), op.sym));
                 }
             }
             slot_wide = fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n;
@@ -1027,6 +1033,9 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                                 tt.a_z = static_cast<unsigned short>(p.a_z);
                                 tt.b_z = static_cast<unsigned short>(p.b_z);
                                 tt.bibj = (static_cast<unsigned>(bi) << 16) | static_cast<unsigned>(bj);
+                                // wide tile of a symmetric output: a lower first half is skipped
+                                if (op.sym && tw > tile_n && bi > bj * (tw / tile_n))
+                                    tt.kf |= static_cast<unsigned>(TILE_LOWER0) << 24;
                                 tt.mat = static_cast<unsigned>(mi);
                                 tt.need = chained ? kTileArrivals * mat_tiles_done[mi] : 0u;
                                 ltiles.push_back({tt, K});

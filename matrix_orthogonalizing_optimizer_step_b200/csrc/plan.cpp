@@ -654,9 +654,11 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     // A launch takes them when its FLOP-weighted K is at least kWideMinK
     // (shorter, the exposed epilogue costs more than the bytes save) and its
     // wide tiles compute at most kWideMaxArea times the area of its 256-wide
-    // ones, K-weighted.  Chained launches keep 256 x 256 tiles and the
-    // double-buffered accumulators.
-    constexpr double kWideMinK = 3072.0, kWideMaxArea = 1.08;
+    // ones, K-weighted, and it has at least kWideMinRounds wide tiles per
+    // resident CTA pair (with fewer, the epilogues that no longer overlap and
+    // the last round's tail dominate).  Chained launches keep 256 x 256 tiles
+    // and the double-buffered accumulators.
+    constexpr double kWideMinK = 3072.0, kWideMaxArea = 1.08, kWideMinRounds = 4.0;
     const bool wide = !f32 && !chained && wide_tiles_allowed();
     // 256-column blocks computed by the 256 x tw tiles of an M x N output
     // (symmetric: tiles wholly below the diagonal are left out, and a wide
@@ -669,6 +671,13 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                 if (sym && bi * tile_m > bj * tw + tw - 1) continue;
                 n += (sym && per > 1 && bi > bj * per) ? per - 1 : per;
             }
+        return n;
+    };
+    auto tile_count = [&](int M, int N, int tw, bool sym) {
+        long long n = 0;
+        for (int bi = 0; bi < (M + tile_m - 1) / tile_m; ++bi)
+            for (int bj = 0; bj < (N + tw - 1) / tw; ++bj)
+                if (!(sym && bi * tile_m > bj * tw + tw - 1)) ++n;
         return n;
     };
     const unsigned long long wait_ns = wait_limit_ns();
@@ -873,7 +882,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     for (size_t si = 0; si < nslots; ++si) {
         bool slot_wide = false;
         if (wide) {
-            double fk = 0.0, fsum = 0.0, area_w = 0.0, area_n = 0.0;
+            double fk = 0.0, fsum = 0.0, area_w = 0.0, area_n = 0.0, tiles_w = 0.0;
             for (const Group& g : groups) {
                 if (si >= g.slots.size()) continue;
                 for (const OpDesc& op : g.slots[si]) {
@@ -886,9 +895,12 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                     const double kw = static_cast<double>(K) * static_cast<double>(g.mats.size());
                     area_n += kw * static_cast<double>(block_count(M, N, tile_n, op.sym));
                     area_w += kw * static_cast<double>(block_count(M, N, gemm_tc_wide_tile_n(), op.sym));
+                    tiles_w += static_cast<double>(g.mats.size()) *
+                               static_cast<double>(tile_count(M, N, gemm_tc_wide_tile_n(), op.sym));
                 }
             }
-            slot_wide = fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n;
+            slot_wide = fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n &&
+                        tiles_w >= kWideMinRounds * std::max(1, max_pairs);
         }
         const int slot_tile_n = slot_wide ? gemm_tc_wide_tile_n() : tile_n;
         LaunchRec lr;

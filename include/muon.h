@@ -58,6 +58,8 @@
  *    MUON_CHAIN_LAUNCH / MUON_SLOT_LAUNCHES  force one launch for the whole
  *                        Newton-Schulz chain / one launch per chain slot
  *    MUON_TMA_STORE=0    plain per-lane stores in the GEMM epilogue
+ *    MUON_TILE_N=256|512 per-slot launches use 256-wide tiles only / 512-wide
+ *                        tiles always (default: chosen per launch)
  *    MUON_DEBUG_CANARY=1 every workspace region is followed by a 1 KB guard
  *                        of a fixed byte pattern; after each call's launches
  *                        a check kernel compares every guard with it (and

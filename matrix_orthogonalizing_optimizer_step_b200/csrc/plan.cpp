@@ -85,11 +85,15 @@ int fault_mode() {
     return FAULT_NONE;
 }
 
-// MUON_TILE_N=256 (read when a plan is built): persistent launches keep
-// 256-wide tiles instead of 512-wide ones.
-bool wide_tiles_allowed() {
+// MUON_TILE_N (read when a plan is built): 256 = persistent launches keep
+// 256-wide tiles; 512 = every persistent launch takes 512-wide tiles (tests of
+// the wide instance on any shape); unset = chosen per launch.
+enum { TILES_AUTO = 0, TILES_NARROW = 1, TILES_WIDE = 2 };
+int tile_mode() {
     const char* v = std::getenv("MUON_TILE_N");
-    return !(v && std::atoi(v) == 256);
+    if (v && std::atoi(v) == 256) return TILES_NARROW;
+    if (v && std::atoi(v) == 512) return TILES_WIDE;
+    return TILES_AUTO;
 }
 
 bool canary_mode() {
@@ -386,7 +390,7 @@ static std::vector<long long> make_key(const PlanRequest& rq) {
     for (int si : rq.sched) k.push_back(si);
     k.push_back(fault_mode());
     k.push_back(canary_mode() ? 1 : 0);
-    k.push_back(wide_tiles_allowed() ? 1 : 0);
+    k.push_back(tile_mode());
     k.push_back(static_cast<long long>(wait_limit_ns()));
     for (size_t i = 0; i < rq.rows.size(); ++i) {
         k.push_back(rq.rows[i]);
@@ -659,7 +663,7 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
     // the last round's tail dominate).  Chained launches keep 256 x 256 tiles
     // and the double-buffered accumulators.
     constexpr double kWideMinK = 3072.0, kWideMaxArea = 1.08, kWideMinRounds = 4.0;
-    const bool wide = !f32 && !chained && wide_tiles_allowed();
+    const bool wide = !f32 && !chained && tile_mode() != TILES_NARROW;
     // 256-column blocks computed by the 256 x tw tiles of an M x N output
     // (symmetric: tiles wholly below the diagonal are left out, and a wide
     // tile's lower first half is not computed)
@@ -899,8 +903,9 @@ int Plan::build(const PlanRequest& rq, DeviceStatus* status, int num_sms, cudaSt
                                static_cast<double>(tile_count(M, N, gemm_tc_wide_tile_n(), op.sym));
                 }
             }
-            slot_wide = fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n &&
-                        tiles_w >= kWideMinRounds * std::max(1, max_pairs);
+            slot_wide = tile_mode() == TILES_WIDE ||
+                        (fsum > 0.0 && fk >= kWideMinK * fsum && area_w <= kWideMaxArea * area_n &&
+                         tiles_w >= kWideMinRounds * std::max(1, max_pairs));
         }
         const int slot_tile_n = slot_wide ? gemm_tc_wide_tile_n() : tile_n;
         LaunchRec lr;

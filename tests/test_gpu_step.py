@@ -394,3 +394,35 @@ def test_llama8b_set_full_size_sampled():
     """Workload 5 (Llama-8B Muon set, 224 matrices, 6.98 G elements) at full
     size: one matrix of each of the four shapes against the oracle."""
     _full_size_sampled(5, [0, 2, 4, 6])
+
+
+@pytest.mark.parametrize("form", ["auto", "standard", "gram"])
+def test_wide_tiles_bitwise_equal_to_256_wide(form, monkeypatch):
+    """The 512-wide tile instance (forced on every per-slot launch) against
+    256-wide tiles: ragged N (not a multiple of 512), transposed matrices,
+    symmetric outputs whose wide tiles skip a lower first half, n x n
+    products of several 256-blocks.  Each output element is the same MMA
+    sequence and epilogue either way, so the results are bitwise equal."""
+    shapes = [(768, 2304), (3072, 768), (1000, 1000), (520, 1544), (1300, 700), (200, 712), (37, 91)]
+
+    def run(tile_n):
+        monkeypatch.setenv("MUON_SLOT_LAUNCHES", "1")
+        monkeypatch.setenv("MUON_TILE_N", tile_n)
+        mo.muon_release_workspace()
+        mo.muon_set_config(mode=form)
+        W, G, M = _make_set(shapes, 1700)
+        for _ in range(2):
+            mo.muon_step(W, G, M, mu=0.95, nesterov=True, lr=0.02)
+        X = torch.stack([wl.make_single(1300, 1544, 1750 + j, "gaussian", DEV, "bf16") for j in range(2)])
+        mo.muon_orthogonalize(X, steps=5, mode=form)
+        torch.cuda.synchronize()
+        out = [t.clone() for t in W + M + [X]]
+        monkeypatch.delenv("MUON_TILE_N")
+        monkeypatch.delenv("MUON_SLOT_LAUNCHES")
+        mo.muon_release_workspace()
+        return out
+
+    ref = run("256")
+    got = run("512")
+    for a, b in zip(ref, got):
+        assert torch.equal(a, b)
